@@ -1,0 +1,184 @@
+/*
+ * i8lt.h — C ABI of the B200 (sm_100a) LLM.int8() Linear8bitLt forward library.
+ *
+ * The operation is the mixed int8/fp16 decomposition of
+ * "`bitsandbytes` - `Linear8bitLt` integration into `transformers` models"
+ * (HF transformers PR #17901, section "About the mixed quantization method in
+ * few words": outlier features go through fp16, the rest through int8), built
+ * from the ops named in "LLM.int8() Refactoring: Part 1" (bitsandbytes PR
+ * #1401): the fused calibration + quantisation kernel of section "Improved
+ * kernels for inference" (int8_vectorwise_quant), the int8 GEMM and dequant
+ * ops of section "Deprecations" (igemmlt -> int8_linear_matmul, mm_dequant ->
+ * int8_mm_dequant), and the int8 dequantize op of section "Next steps".
+ *
+ * Conventions shared by every entry point
+ *   - All matrices are dense row-major.  X / out / bias / W hold IEEE binary16
+ *     bits (i8_half); CA / CB hold signed int8 codes in [-127, 127]; SCA / SCB
+ *     are fp32 row absmax scales; C is int32.
+ *   - Every pointer is a DEVICE pointer unless stated otherwise.  The caller
+ *     owns every buffer: the library never allocates or frees memory, keeps no
+ *     mutable global state, and may be called concurrently on different
+ *     streams as long as the calls do not share output or workspace buffers.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and is asynchronous: I8_OK means "arguments valid and
+ *     kernels enqueued".  Nothing synchronises the host except i8_read_status.
+ *   - Argument errors are returned before anything is enqueued.  Matrix
+ *     pointers must be 16-byte aligned and K must be a multiple of 16 (the TMA
+ *     row-stride rule); M, N, K must be > 0.  The threshold must be finite and
+ *     >= 0; 0 turns outlier handling off.
+ *   - Errors found on the device (more outlier columns than the workspace
+ *     holds, a pipeline wait that ran past its time limit) are written to a
+ *     status word in device memory and read back with i8_read_status.
+ *   - Numerics: quantisation rounds x * fl32(127 / absmax) to nearest-even in
+ *     fp32; the int8 product is exact in int32; dequantisation is fp32 and the
+ *     result is rounded once to fp16.
+ */
+#ifndef I8LT_H_
+#define I8LT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define I8_API __attribute__((visibility("default")))
+#else
+#define I8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t i8_half;          /* IEEE 754 binary16 bit pattern */
+typedef struct CUstream_st* i8_stream_t;   /* identical to cudaStream_t */
+
+typedef enum {
+  I8_OK = 0,
+  I8_ERR_INVALID_ARG = 1,        /* null pointer, non-positive size, bad threshold */
+  I8_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 16 != 0, misaligned pointer, size limits */
+  I8_ERR_WORKSPACE = 3,          /* workspace too small or misaligned */
+  I8_ERR_CUDA = 4,               /* a CUDA runtime / driver call failed */
+  I8_ERR_TIMEOUT = 5,            /* device: a pipeline wait ran past its time limit */
+  I8_ERR_OUTLIER_OVERFLOW = 6    /* device: more outlier columns than max_outlier_cols */
+} i8_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+I8_API const char* i8_status_string(i8_status s);
+
+/*
+ * i8_quantize_rowwise — fused row-wise calibration, int8 quantisation and
+ * outlier-column detection ("LLM.int8() Refactoring: Part 1", section
+ * "Improved kernels for inference": int8_vectorwise_quant; outlier columns are
+ * the `state.idx` of the review of bitsandbytes/autograd/_functions.py).
+ *
+ *   X       [M, K] fp16 input (tokens x features).
+ *   CA      [M, K] int8 output codes.
+ *   SCA     [M]    fp32 output: per row, the max |x| over the elements whose
+ *                  magnitude is below `threshold` (all elements if it is 0).
+ *   bitmap  [ceil(K/32)] uint32 output, required when threshold > 0 (may be
+ *           NULL otherwise): bit (j % 32) of word j / 32 is set iff some
+ *           element of column j has |x| >= threshold.  Overwritten.
+ * Codes: CA = clamp(rne(x * fl32(127/SCA)), -127, 127), 0 when SCA == 0, and
+ * every outlier column of CA is 0 in every row (that column belongs to the
+ * fp16 path).  Uses the caller's `bitmap` as its only scratch.
+ */
+I8_API i8_status i8_quantize_rowwise(const i8_half* X, int M, int K, float threshold,
+                              int8_t* CA, float* SCA, uint32_t* bitmap,
+                              i8_stream_t stream);
+
+/*
+ * i8_outlier_columns — compact an outlier bitmap into the sorted list of
+ * outlier column indices (the `state.idx` of "LLM.int8() Refactoring: Part 1",
+ * review of bitsandbytes/autograd/_functions.py).
+ *   bitmap [ceil(K/32)] uint32 input; idx [max_cols] int32 output (ascending);
+ *   count  one int32 output = number of outlier columns found (may exceed
+ *   max_cols; only the first max_cols indices are written).
+ */
+I8_API i8_status i8_outlier_columns(const uint32_t* bitmap, int K, int32_t* idx,
+                             int max_cols, int32_t* count, i8_stream_t stream);
+
+/*
+ * i8_int8_linear_matmul — C = A . B^T exactly, int8 x int8 -> int32
+ * ("LLM.int8() Refactoring: Part 1", section "Deprecations": igemmlt becomes
+ * int8_linear_matmul; row-major operands).
+ *   A [M, K] int8, B [N, K] int8 (both K-contiguous), C [M, N] int32 output.
+ * |C| <= 127*128*K always fits int32 for K <= 131072.
+ */
+I8_API i8_status i8_int8_linear_matmul(const int8_t* A, const int8_t* B, int M, int N, int K,
+                                int32_t* C, i8_stream_t stream);
+
+/*
+ * i8_int8_mm_dequant — out = fp16(C * SCA[i] * SCB[n] / 127^2 + bias[n])
+ * ("LLM.int8() Refactoring: Part 1", section "Deprecations": mm_dequant
+ * becomes int8_mm_dequant; commit "New naive mm_dequant kernel for row-major").
+ *   C [M, N] int32, SCA [M] fp32, SCB [N] fp32, bias [N] fp16 or NULL,
+ *   out [M, N] fp16 output.
+ */
+I8_API i8_status i8_int8_mm_dequant(const int32_t* C, const float* SCA, const float* SCB,
+                             const i8_half* bias, int M, int N, i8_half* out,
+                             i8_stream_t stream);
+
+/*
+ * i8_dequant — int8 weight back to fp16: W = fp16(CB * SCB[n] / 127)
+ * ("LLM.int8() Refactoring: Part 1", section "Next steps": int8 dequantize op).
+ *   CB [N, K] int8, SCB [N] fp32, W [N, K] fp16 output.
+ */
+I8_API i8_status i8_dequant(const int8_t* CB, const float* SCB, int N, int K, i8_half* W,
+                     i8_stream_t stream);
+
+/*
+ * Workspace bytes i8_linear8bit_forward needs for these sizes.  The workspace
+ * is caller-owned device memory, 256-byte aligned, that holds CA, SCA, the
+ * outlier bitmap / index list, the gathered fp16 outlier operands and the
+ * status word.  Returns 0 for invalid sizes.
+ */
+I8_API size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_cols);
+
+/*
+ * i8_linear8bit_forward — LLM.int8() Linear8bitLt forward
+ * ("`bitsandbytes` - `Linear8bitLt` integration into `transformers` models",
+ * section "About the mixed quantization method in few words"):
+ *
+ *   out[i, n] = fp16( C[i,n] * SCA[i] * SCB[n] / 127^2 + bias[n]
+ *                     + (SCB[n] / 127) * sum_{j in O} X[i, j] * CB[n, j] )
+ *
+ * where CA, SCA, O come from i8_quantize_rowwise(X, threshold) and
+ * C = CA . CB^T.  X [M, K] fp16; CB [N, K] int8 and SCB [N] fp32 from
+ * i8_quantize_rowwise(W, threshold = 0); bias [N] fp16 or NULL; out [M, N]
+ * fp16 output.  The outlier term runs on the fp16 tensor-core path; O is read
+ * on the device, so the call never waits for the host.
+ *   workspace / workspace_bytes: see i8_linear8bit_workspace_size.
+ *   max_outlier_cols: capacity for |O|; if more columns reach the threshold,
+ *   the status word becomes I8_ERR_OUTLIER_OVERFLOW and out is unspecified.
+ * Enqueues a small memset plus four kernels (quantise, outlier prepare,
+ * tensor-core GEMM with fused dequant epilogue; a split-K reduction kernel is
+ * used for M <= 16).
+ */
+I8_API i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const float* SCB,
+                                const i8_half* bias, int M, int N, int K, float threshold,
+                                i8_half* out, void* workspace, size_t workspace_bytes,
+                                int max_outlier_cols, i8_stream_t stream);
+
+/*
+ * i8_read_status — synchronise `stream` and return the device status word of
+ * the last i8_linear8bit_forward that used `workspace` (I8_OK, I8_ERR_TIMEOUT
+ * or I8_ERR_OUTLIER_OVERFLOW), or I8_ERR_CUDA if the synchronisation failed.
+ * `count` (host pointer, may be NULL) receives the number of outlier columns
+ * that call found.
+ */
+I8_API i8_status i8_read_status(const void* workspace, int32_t* count, i8_stream_t stream);
+
+/*
+ * i8_selftest_bounded_wait — failure-detection self test.  Launches one block
+ * that waits on a shared-memory barrier that nothing ever completes, with the
+ * same bounded-wait routine the GEMM pipeline uses and a limit of
+ * `limit_ns` nanoseconds (1 ms .. 10 s).  The kernel gives up, writes
+ * I8_ERR_TIMEOUT to *status (device uint32) and returns; nothing hangs.
+ */
+I8_API i8_status i8_selftest_bounded_wait(uint32_t* status, uint64_t limit_ns, i8_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* I8LT_H_ */

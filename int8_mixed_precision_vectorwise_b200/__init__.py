@@ -1,0 +1,22 @@
+"""LLM.int8() Linear8bitLt forward for B200 (sm_100a).
+
+The compute path is the CUDA library ``libi8lt.so`` (C ABI in
+``include/i8lt.h``); this package is a thin ctypes binding over it with the
+same entry-point names.  PyTorch supplies device memory and streams only.
+"""
+
+from ._binding import (  # noqa: F401
+    I8Error,
+    LIB_PATH,
+    STATUS,
+    i8_dequant,
+    i8_int8_linear_matmul,
+    i8_int8_mm_dequant,
+    i8_linear8bit_forward,
+    i8_linear8bit_workspace_size,
+    i8_outlier_columns,
+    i8_quantize_rowwise,
+    i8_read_status,
+    i8_selftest_bounded_wait,
+    lib,
+)

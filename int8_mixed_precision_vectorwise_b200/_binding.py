@@ -1,0 +1,218 @@
+"""ctypes binding of ``libi8lt.so`` (the C ABI in ``include/i8lt.h``).
+
+Argument marshalling only: every function checks dtypes / devices / shapes of
+torch tensors, allocates missing outputs with torch, and forwards raw device
+pointers plus the current CUDA stream to the library.  All arithmetic runs in
+the library's CUDA kernels; there is no fallback.  If the library is missing
+or cannot be loaded, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libi8lt.so")
+
+STATUS = {
+    0: "I8_OK",
+    1: "I8_ERR_INVALID_ARG",
+    2: "I8_ERR_UNSUPPORTED_SHAPE",
+    3: "I8_ERR_WORKSPACE",
+    4: "I8_ERR_CUDA",
+    5: "I8_ERR_TIMEOUT",
+    6: "I8_ERR_OUTLIER_OVERFLOW",
+}
+I8_OK = 0
+
+EXPORTS = (
+    "i8_status_string", "i8_quantize_rowwise", "i8_outlier_columns", "i8_int8_linear_matmul",
+    "i8_int8_mm_dequant", "i8_dequant", "i8_linear8bit_workspace_size", "i8_linear8bit_forward",
+    "i8_read_status", "i8_selftest_bounded_wait",
+)
+
+
+class I8Error(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+_lock = threading.Lock()
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_S = ctypes.c_size_t
+
+
+def _declare(lib):
+    sig = {
+        "i8_status_string": (ctypes.c_char_p, [_I]),
+        "i8_quantize_rowwise": (_I, [_P, _I, _I, _F, _P, _P, _P, _P]),
+        "i8_outlier_columns": (_I, [_P, _I, _P, _I, _P, _P]),
+        "i8_int8_linear_matmul": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+        "i8_int8_mm_dequant": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
+        "i8_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
+        "i8_linear8bit_workspace_size": (_S, [_I, _I, _I, _I]),
+        "i8_linear8bit_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
+        "i8_read_status": (_I, [_P, _P, _P]),
+        "i8_selftest_bounded_wait": (_I, [_P, ctypes.c_uint64, _P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+def lib():
+    """The loaded library (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"{LIB_PATH} is missing: build it with "
+                        "`python -m int8_mixed_precision_vectorwise_b200.build`")
+                _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def _check(fn: str, code: int):
+    if code != I8_OK:
+        raise I8Error(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D")
+
+
+# ----------------------------------------------------------------- entry points
+def i8_quantize_rowwise(X, threshold: float = 0.0, CA=None, SCA=None, bitmap=None):
+    """Fused row absmax + int8 quantisation + outlier bitmap.  Returns (CA, SCA, bitmap)."""
+    _need(X, torch.float16, "X", 2)
+    M, K = X.shape
+    dev = X.device
+    CA = torch.empty((M, K), dtype=torch.int8, device=dev) if CA is None else CA
+    SCA = torch.empty((M,), dtype=torch.float32, device=dev) if SCA is None else SCA
+    if threshold > 0 and bitmap is None:
+        bitmap = torch.empty(((K + 31) // 32,), dtype=torch.int32, device=dev)
+    _check("i8_quantize_rowwise", lib().i8_quantize_rowwise(
+        _ptr(X), M, K, float(threshold), _ptr(CA), _ptr(SCA), _ptr(bitmap), _stream(dev)))
+    return CA, SCA, bitmap
+
+
+def i8_outlier_columns(bitmap, K: int, max_cols: int, idx=None, count=None):
+    """Sorted outlier column list from a bitmap.  Returns (idx[max_cols], count[1]) on device."""
+    _need(bitmap, torch.int32, "bitmap", 1)
+    dev = bitmap.device
+    idx = torch.empty((max(max_cols, 1),), dtype=torch.int32, device=dev) if idx is None else idx
+    count = torch.empty((1,), dtype=torch.int32, device=dev) if count is None else count
+    _check("i8_outlier_columns", lib().i8_outlier_columns(
+        _ptr(bitmap), K, _ptr(idx), max_cols, _ptr(count), _stream(dev)))
+    return idx, count
+
+
+def i8_int8_linear_matmul(A, B, C=None):
+    """C = A . B^T, int8 x int8 -> int32 (exact)."""
+    _need(A, torch.int8, "A", 2)
+    _need(B, torch.int8, "B", 2)
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("A and B must share K")
+    C = torch.empty((M, N), dtype=torch.int32, device=A.device) if C is None else C
+    _check("i8_int8_linear_matmul", lib().i8_int8_linear_matmul(
+        _ptr(A), _ptr(B), M, N, K, _ptr(C), _stream(A.device)))
+    return C
+
+
+def i8_int8_mm_dequant(C, SCA, SCB, bias=None, out=None):
+    """out = fp16(C * SCA[i] * SCB[n] / 127^2 + bias[n])."""
+    _need(C, torch.int32, "C", 2)
+    _need(SCA, torch.float32, "SCA", 1)
+    _need(SCB, torch.float32, "SCB", 1)
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    M, N = C.shape
+    out = torch.empty((M, N), dtype=torch.float16, device=C.device) if out is None else out
+    _check("i8_int8_mm_dequant", lib().i8_int8_mm_dequant(
+        _ptr(C), _ptr(SCA), _ptr(SCB), _ptr(bias), M, N, _ptr(out), _stream(C.device)))
+    return out
+
+
+def i8_dequant(CB, SCB, W=None):
+    """W = fp16(CB * SCB[n] / 127)."""
+    _need(CB, torch.int8, "CB", 2)
+    _need(SCB, torch.float32, "SCB", 1)
+    N, K = CB.shape
+    W = torch.empty((N, K), dtype=torch.float16, device=CB.device) if W is None else W
+    _check("i8_dequant", lib().i8_dequant(_ptr(CB), _ptr(SCB), N, K, _ptr(W), _stream(CB.device)))
+    return W
+
+
+def i8_linear8bit_workspace_size(M: int, N: int, K: int, max_outlier_cols: int) -> int:
+    n = lib().i8_linear8bit_workspace_size(M, N, K, max_outlier_cols)
+    if n == 0:
+        raise I8Error("i8_linear8bit_workspace_size", 1)
+    return int(n)
+
+
+def i8_linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, out=None, workspace=None,
+                          max_outlier_cols: int = 256):
+    """LLM.int8() Linear8bitLt forward.  Returns (out, workspace)."""
+    _need(X, torch.float16, "X", 2)
+    _need(CB, torch.int8, "CB", 2)
+    _need(SCB, torch.float32, "SCB", 1)
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    M, K = X.shape
+    N = CB.shape[0]
+    if CB.shape[1] != K:
+        raise ValueError("X and CB must share K")
+    dev = X.device
+    need = i8_linear8bit_workspace_size(M, N, K, max_outlier_cols)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    out = torch.empty((M, N), dtype=torch.float16, device=dev) if out is None else out
+    _check("i8_linear8bit_forward", lib().i8_linear8bit_forward(
+        _ptr(X), _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out),
+        _ptr(workspace), workspace.numel(), max_outlier_cols, _stream(dev)))
+    return out, workspace
+
+
+def i8_read_status(workspace):
+    """Synchronise the current stream; returns (status_code, outlier_count) of the last forward."""
+    cnt = ctypes.c_int32(0)
+    code = lib().i8_read_status(_ptr(workspace), ctypes.byref(cnt), _stream(workspace.device))
+    return int(code), int(cnt.value)
+
+
+def i8_selftest_bounded_wait(status, limit_ns: int):
+    _need(status, torch.int32, "status", 1)
+    _check("i8_selftest_bounded_wait", lib().i8_selftest_bounded_wait(
+        _ptr(status), int(limit_ns), _stream(status.device)))
+    return status

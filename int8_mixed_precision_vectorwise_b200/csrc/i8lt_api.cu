@@ -1,0 +1,302 @@
+// C ABI of the library (declared in include/i8lt.h): argument validation,
+// workspace layout, TMA tensor-map encoding and kernel launches.  Every check
+// that can fail on the host runs before any CUDA call, so argument errors are
+// reported without touching the device.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/i8lt.h"
+#include "kernels.cuh"
+
+namespace {
+
+using i8lt::GemmArgs;
+
+constexpr int kMaxOutlierCap = 8192;                   // shared-memory index list of the prepare kernel
+constexpr uint64_t kWaitLimitNs = 2000000000ull;       // 2 s bound on every pipeline wait
+constexpr size_t kHdrBytes = 256;                      // status, used count, total count
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t hdr, bitmap, idx, sca, ca, xo, wo, total;
+  int ld_o;  // row stride (fp16 elements) of the gathered outlier operands
+};
+
+bool ws_layout(int M, int N, int K, int cap, WsLayout* L) {
+  if (M <= 0 || N <= 0 || K <= 0 || cap < 0) return false;
+  size_t off = 0;
+  L->hdr = off;
+  off += kHdrBytes;
+  L->bitmap = off;
+  off += align256(static_cast<size_t>((K + 31) / 32) * 4);
+  L->idx = off;
+  off += align256(static_cast<size_t>(cap > 0 ? cap : 1) * 4);
+  L->sca = off;
+  off += align256(static_cast<size_t>(M) * 4);
+  L->ca = off;
+  off += align256(static_cast<size_t>(M) * K);
+  L->ld_o = cap > 0 ? ((cap + 63) / 64) * 64 : 0;
+  L->xo = off;
+  off += align256(static_cast<size_t>(M) * L->ld_o * 2);
+  L->wo = off;
+  off += align256(static_cast<size_t>(N) * L->ld_o * 2);
+  L->total = off;
+  return true;
+}
+
+// --------------------------------------------------------------- driver entry point
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major [rows, inner] matrix, boxes of box_inner x box_rows elements, 128B swizzle.
+bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+inline i8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? I8_OK : I8_ERR_CUDA; }
+
+i8_status check_threshold(float t) {
+  if (!std::isfinite(t) || t < 0.f) return I8_ERR_INVALID_ARG;
+  return I8_OK;
+}
+
+// Shape/pointer rules shared by the GEMM entry points.
+i8_status check_gemm_operands(const void* A, const void* B, int M, int N, int K) {
+  if (!A || !B) return I8_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > (1 << 17)) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(A) || !aligned16(B)) return I8_ERR_UNSUPPORTED_SHAPE;
+  return I8_OK;
+}
+
+i8_status run_gemm(const int8_t* A, const int8_t* B, int M, int N, int K, const GemmArgs& args, bool raw,
+                   const __half* XO, const __half* WO, int ld_o, cudaStream_t st) {
+  CUtensorMap tmA, tmB, tmXO, tmWO;
+  std::memset(&tmXO, 0, sizeof(tmXO));
+  std::memset(&tmWO, 0, sizeof(tmWO));
+  if (!encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, i8lt::kGemmBKBytes, i8lt::kGemmBM) ||
+      !encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, i8lt::kGemmBKBytes, i8lt::kGemmBN))
+    return I8_ERR_CUDA;
+  if (XO != nullptr && WO != nullptr && ld_o > 0) {
+    if (!encode_2d(&tmXO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, XO, ld_o, M, static_cast<uint64_t>(ld_o) * 2, 64,
+                   i8lt::kGemmBM) ||
+        !encode_2d(&tmWO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, WO, ld_o, N, static_cast<uint64_t>(ld_o) * 2, 64,
+                   i8lt::kGemmBN))
+      return I8_ERR_CUDA;
+  }
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_gemm(tmA, tmB, tmXO, tmWO, args, raw, sms, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* i8_status_string(i8_status s) {
+  switch (s) {
+    case I8_OK: return "I8_OK";
+    case I8_ERR_INVALID_ARG: return "I8_ERR_INVALID_ARG";
+    case I8_ERR_UNSUPPORTED_SHAPE: return "I8_ERR_UNSUPPORTED_SHAPE";
+    case I8_ERR_WORKSPACE: return "I8_ERR_WORKSPACE";
+    case I8_ERR_CUDA: return "I8_ERR_CUDA";
+    case I8_ERR_TIMEOUT: return "I8_ERR_TIMEOUT";
+    case I8_ERR_OUTLIER_OVERFLOW: return "I8_ERR_OUTLIER_OVERFLOW";
+  }
+  return "I8_ERR_UNKNOWN";
+}
+
+i8_status i8_quantize_rowwise(const i8_half* X, int M, int K, float threshold, int8_t* CA, float* SCA,
+                              uint32_t* bitmap, i8_stream_t stream) {
+  if (!X || !CA || !SCA) return I8_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (check_threshold(threshold) != I8_OK) return I8_ERR_INVALID_ARG;
+  if (threshold > 0.f && !bitmap) return I8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(CA)) return I8_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const __half* Xh = reinterpret_cast<const __half*>(X);
+  if (threshold > 0.f) {
+    if (cudaMemsetAsync(bitmap, 0, static_cast<size_t>((K + 31) / 32) * 4, st) != cudaSuccess) return I8_ERR_CUDA;
+  }
+  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, threshold > 0.f ? bitmap : nullptr, st));
+  if (s != I8_OK || threshold == 0.f) return s;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_zero_outlier_cols(bitmap, M, K, CA, sms, st));
+}
+
+i8_status i8_outlier_columns(const uint32_t* bitmap, int K, int32_t* idx, int max_cols, int32_t* count,
+                             i8_stream_t stream) {
+  if (!bitmap || !count || K <= 0 || max_cols < 0) return I8_ERR_INVALID_ARG;
+  if (max_cols > 0 && !idx) return I8_ERR_INVALID_ARG;
+  if (max_cols > kMaxOutlierCap) return I8_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_outlier_prepare(bitmap, K, max_cols, count, nullptr, idx, nullptr, nullptr,
+                                                  nullptr, 0, nullptr, nullptr, 0, nullptr, 0, sms,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_int8_linear_matmul(const int8_t* A, const int8_t* B, int M, int N, int K, int32_t* C,
+                                i8_stream_t stream) {
+  i8_status s = check_gemm_operands(A, B, M, N, K);
+  if (s != I8_OK) return s;
+  if (!C) return I8_ERR_INVALID_ARG;
+  if (!aligned16(C)) return I8_ERR_UNSUPPORTED_SHAPE;
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.C = C;
+  a.wait_limit_ns = kWaitLimitNs;
+  return run_gemm(A, B, M, N, K, a, true, nullptr, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+i8_status i8_int8_mm_dequant(const int32_t* C, const float* SCA, const float* SCB, const i8_half* bias, int M,
+                             int N, i8_half* out, i8_stream_t stream) {
+  if (!C || !SCA || !SCB || !out) return I8_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0) return I8_ERR_INVALID_ARG;
+  if (!aligned16(C) || !aligned16(SCB) || !aligned16(out) || (bias && !aligned16(bias)))
+    return I8_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_mm_dequant(C, SCA, SCB, reinterpret_cast<const __half*>(bias), M, N,
+                                             reinterpret_cast<__half*>(out), sms,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_dequant(const int8_t* CB, const float* SCB, int N, int K, i8_half* W, i8_stream_t stream) {
+  if (!CB || !SCB || !W) return I8_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (K % 16 != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(CB) || !aligned16(W)) return I8_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_dequant(CB, SCB, N, K, reinterpret_cast<__half*>(W), sms,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_cols) {
+  WsLayout L;
+  if (max_outlier_cols > kMaxOutlierCap || !ws_layout(M, N, K, max_outlier_cols, &L)) return 0;
+  return L.total;
+}
+
+i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const float* SCB, const i8_half* bias, int M,
+                                int N, int K, float threshold, i8_half* out, void* workspace,
+                                size_t workspace_bytes, int max_outlier_cols, i8_stream_t stream) {
+  if (!X || !out || !workspace) return I8_ERR_INVALID_ARG;
+  i8_status s = check_gemm_operands(X, CB, M, N, K);
+  if (s != I8_OK) return s;
+  if (!SCB) return I8_ERR_INVALID_ARG;
+  if (check_threshold(threshold) != I8_OK || max_outlier_cols < 0) return I8_ERR_INVALID_ARG;
+  if (max_outlier_cols > kMaxOutlierCap) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(out) || (bias && !aligned16(bias))) return I8_ERR_UNSUPPORTED_SHAPE;
+  WsLayout L;
+  if (!ws_layout(M, N, K, max_outlier_cols, &L)) return I8_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < L.total) return I8_ERR_WORKSPACE;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* hdr = reinterpret_cast<uint32_t*>(ws + L.hdr);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ws + L.bitmap);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* SCA = reinterpret_cast<float*>(ws + L.sca);
+  int8_t* CA = reinterpret_cast<int8_t*>(ws + L.ca);
+  __half* XO = reinterpret_cast<__half*>(ws + L.xo);
+  __half* WO = reinterpret_cast<__half*>(ws + L.wo);
+  const __half* Xh = reinterpret_cast<const __half*>(X);
+  const bool outliers = threshold > 0.f;
+
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  // status word, counts and the bitmap are contiguous: one memset clears them
+  if (cudaMemsetAsync(ws, 0, L.bitmap + static_cast<size_t>((K + 31) / 32) * 4, st) != cudaSuccess)
+    return I8_ERR_CUDA;
+  s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, outliers ? bitmap : nullptr, st));
+  if (s != I8_OK) return s;
+  if (outliers) {
+    const int cap = max_outlier_cols;
+    s = cuda_status(i8lt::launch_outlier_prepare(bitmap, K, cap, reinterpret_cast<int32_t*>(hdr + 2),
+                                                 reinterpret_cast<int32_t*>(hdr + 1), idx, hdr, CA, Xh, M,
+                                                 cap > 0 ? XO : nullptr, CB, N, cap > 0 ? WO : nullptr, L.ld_o,
+                                                 sms, st));
+    if (s != I8_OK) return s;
+  }
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.SCA = SCA;
+  a.SCB = SCB;
+  a.bias = reinterpret_cast<const __half*>(bias);
+  a.out = reinterpret_cast<__half*>(out);
+  a.n_used = (outliers && max_outlier_cols > 0) ? reinterpret_cast<const int32_t*>(hdr + 1) : nullptr;
+  a.out_cap = max_outlier_cols;
+  a.status = hdr;
+  a.wait_limit_ns = kWaitLimitNs;
+  const bool with_o = outliers && max_outlier_cols > 0;
+  return run_gemm(CA, CB, M, N, K, a, false, with_o ? XO : nullptr, with_o ? WO : nullptr, L.ld_o, st);
+}
+
+i8_status i8_read_status(const void* workspace, int32_t* count, i8_stream_t stream) {
+  if (!workspace) return I8_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t h[3] = {0, 0, 0};
+  if (cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return I8_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return I8_ERR_CUDA;
+  if (count) *count = static_cast<int32_t>(h[2]);
+  return static_cast<i8_status>(h[0]);
+}
+
+i8_status i8_selftest_bounded_wait(uint32_t* status, uint64_t limit_ns, i8_stream_t stream) {
+  if (!status) return I8_ERR_INVALID_ARG;
+  if (limit_ns < 1000000ull || limit_ns > 10000000000ull) return I8_ERR_INVALID_ARG;
+  return cuda_status(i8lt::launch_selftest_wait(status, limit_ns, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

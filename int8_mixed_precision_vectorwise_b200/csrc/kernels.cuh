@@ -1,0 +1,51 @@
+// Host-side launchers of the library's kernels (all enqueue on the given stream).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace i8lt {
+
+cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
+                              cudaStream_t st);
+cudaError_t launch_zero_outlier_cols(const uint32_t* bitmap, int M, int K, int8_t* CA, int num_sms,
+                                     cudaStream_t st);
+cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32_t* total_out, int32_t* used_out,
+                                   int32_t* idx_out, uint32_t* status, int8_t* CA, const __half* X, int M,
+                                   __half* XO, const int8_t* CB, int N, __half* WO, int ld_o, int num_sms,
+                                   cudaStream_t st);
+cudaError_t launch_mm_dequant(const int32_t* C, const float* SCA, const float* SCB, const __half* bias, int M,
+                              int N, __half* out, int num_sms, cudaStream_t st);
+cudaError_t launch_dequant(const int8_t* CB, const float* SCB, int N, int K, __half* W, int num_sms,
+                           cudaStream_t st);
+
+// Tensor-core GEMM (tcgen05, TMA-fed, TMEM accumulators).
+struct GemmArgs {
+  int M, N, K;
+  const float* SCA;        // [M]   (fused mode)
+  const float* SCB;        // [N]   (fused mode)
+  const __half* bias;      // [N] or nullptr
+  __half* out;             // [M, N] fp16 (fused mode)
+  int32_t* C;              // [M, N] int32 (raw mode)
+  const int32_t* n_used;   // device count of gathered outlier columns, or nullptr
+  int out_cap;             // capacity of the gathered outlier operands (columns)
+  uint32_t* status;        // device status word, or nullptr
+  uint64_t wait_limit_ns;  // bound on every pipeline wait
+};
+
+// tmA: CA [M, K] int8; tmB: CB [N, K] int8; tmXO / tmWO: gathered fp16 outlier
+// operands [M, ld] / [N, ld] (unused unless n_used != nullptr).
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmXO,
+                        const CUtensorMap& tmWO, const GemmArgs& a, bool raw_int32, int num_sms, cudaStream_t st);
+
+// Box sizes the tensor maps above must be encoded with.
+constexpr int kGemmBM = 128;       // rows of A per tile
+constexpr int kGemmBN = 256;       // rows of B per tile
+constexpr int kGemmBKBytes = 128;  // bytes of K per pipeline stage
+
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
+
+}  // namespace i8lt

@@ -1,0 +1,282 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bit-exact: int8 codes, fp32 absmax scales, outlier bitmaps / column lists and
+int32 accumulators.  fp16 outputs: |gpu - oracle| <= 1e-2 + 1e-3 * |oracle|
+element by element (the allclose form; 1e-2 alone would reject legitimate one-
+ulp fp16 differences above 16, 1e-3 alone would reject them near 0).
+Every oracle input is generated here or by the oracle itself; nothing the CUDA
+path computed is ever fed to the oracle.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int8_mixed_precision_vectorwise_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 1e-2, 1e-3
+
+
+@pytest.fixture(scope="module")
+def i8():
+    from int8_mixed_precision_vectorwise_b200 import build
+    build.build()
+    import int8_mixed_precision_vectorwise_b200 as m
+    m.lib()
+    return m
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def assert_close(got, ref, what=""):
+    g = np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape
+    d = np.abs(g - r)
+    bad = d > ATOL + RTOL * np.abs(r)
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} out of tolerance; first {tuple(i)} "
+                             f"got {g[tuple(i)]} want {r[tuple(i)]}; max abs {d.max():.3g}")
+
+
+def bitmap_np(t):
+    return host(t).view(np.uint32)
+
+
+def act(M, K, n_out, mag=(20.0, 60.0), seed=0):
+    return wl.activation(wl.BASE_SEED + seed, M, K, n_out, mag)
+
+
+# ------------------------------------------------------------------ quantise
+QSHAPES = [
+    (1, 16, 0.0, 0), (3, 1024, 6.0, 2), (37, 4096, 6.0, 4), (130, 5120, 6.0, 5), (64, 8192, 6.0, 8),
+    (16, 11008, 6.0, 11), (5, 28672, 6.0, 8), (3, 40000, 6.0, 3), (300, 2064, 0.0, 0), (1000, 272, 6.0, 1),
+    (9, 4096, 6.0, 0), (257, 1040, 2.5, 0),
+]
+
+
+@pytest.mark.parametrize("M,K,tau,n_out", QSHAPES)
+def test_quantize_rowwise_bit_exact(i8, M, K, tau, n_out):
+    X, _ = act(M, K, n_out, seed=M + K)
+    CA, SCA, bm = i8.i8_quantize_rowwise(dev(X), tau)
+    rCA, rSCA, rcols = oracle.quantize_rowwise(X, tau)
+    assert np.array_equal(host(CA), rCA)
+    assert np.array_equal(host(SCA).view(np.uint32), rSCA.view(np.uint32))
+    if tau > 0:
+        assert np.array_equal(bitmap_np(bm), oracle.outlier_bitmap(rcols, K))
+
+
+def test_quantize_edge_values(i8):
+    """Exact threshold hits, just-below values, zero rows, rows of outliers only, fp16 extremes."""
+    M, K = 8, 64
+    X = np.zeros((M, K), np.float16)
+    X[0, :] = 1.0
+    X[0, 3] = 6.0                     # exactly at the threshold -> outlier column 3
+    X[1, :] = np.float16(5.99609375)  # just below: no outlier
+    X[2, :] = 0.0                     # zero row
+    X[3, :] = 7.0                     # every column an outlier in this row
+    X[4, :] = np.float16(65504.0)     # fp16 max
+    X[4, 1::2] = -np.float16(0.5)
+    X[5, :] = np.float16(6e-8)        # subnormal
+    X[6, ::3] = np.float16(-2.5)
+    X[7, :] = np.float16(1.5)
+    X[7, 10] = np.float16(-1.5)
+    for tau in (0.0, 6.0, 0.25):
+        CA, SCA, bm = i8.i8_quantize_rowwise(dev(X), tau)
+        rCA, rSCA, rcols = oracle.quantize_rowwise(X, tau)
+        assert np.array_equal(host(CA), rCA), tau
+        assert np.array_equal(host(SCA).view(np.uint32), rSCA.view(np.uint32)), tau
+        if tau > 0:
+            assert np.array_equal(bitmap_np(bm), oracle.outlier_bitmap(rcols, K))
+
+
+@pytest.mark.parametrize("K,n_out,cap", [(4096, 4, 64), (11008, 11, 8), (64, 64, 64), (28672, 0, 16)])
+def test_outlier_columns(i8, K, n_out, cap):
+    X, _ = act(4, K, n_out, seed=K)
+    _, _, bm = i8.i8_quantize_rowwise(dev(X), 6.0)
+    idx, cnt = i8.i8_outlier_columns(bm, K, cap)
+    _, _, rcols = oracle.quantize_rowwise(X, 6.0)
+    assert int(host(cnt)[0]) == len(rcols)
+    k = min(cap, len(rcols))
+    assert host(idx)[:k].tolist() == rcols[:k].tolist()
+
+
+def test_weight_quant_matches_oracle(i8):
+    W = wl.weight(99, 520, 1040)
+    CB, SCB, _ = i8.i8_quantize_rowwise(dev(W), 0.0)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    assert np.array_equal(host(CB), rCB)
+    assert np.array_equal(host(SCB).view(np.uint32), rSCB.view(np.uint32))
+
+
+# ------------------------------------------------------------------ int8 GEMM
+GSHAPES = [(128, 256, 128), (1, 1, 16), (37, 300, 272), (300, 520, 1040), (256, 512, 4096), (513, 257, 160),
+           (129, 1000, 2064), (16, 4096, 28672), (1024, 768, 512)]
+
+
+@pytest.mark.parametrize("M,N,K", GSHAPES)
+def test_int8_linear_matmul_bit_exact(i8, M, N, K):
+    g = np.random.default_rng(M * 7 + N * 3 + K)
+    A = g.integers(-128, 128, size=(M, K), dtype=np.int8)
+    B = g.integers(-128, 128, size=(N, K), dtype=np.int8)
+    A[0, :] = -128
+    B[0, :] = -128
+    C = i8.i8_int8_linear_matmul(dev(A), dev(B))
+    assert np.array_equal(host(C), oracle.int8_linear_matmul(A, B))
+
+
+def test_int8_linear_matmul_repeat_and_stream(i8):
+    g = np.random.default_rng(1)
+    A = g.integers(-127, 128, size=(384, 1024), dtype=np.int8)
+    B = g.integers(-127, 128, size=(640, 1024), dtype=np.int8)
+    ref = oracle.int8_linear_matmul(A, B)
+    s = torch.cuda.Stream()
+    dA, dB = dev(A), dev(B)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        outs = [i8.i8_int8_linear_matmul(dA, dB) for _ in range(3)]
+    s.synchronize()
+    for C in outs:
+        assert np.array_equal(C.cpu().numpy(), ref)
+
+
+# ------------------------------------------------------------------ dequant ops
+@pytest.mark.parametrize("M,N,bias", [(7, 12, True), (33, 1001, False), (256, 4096, True), (1, 3, True)])
+def test_mm_dequant(i8, M, N, bias):
+    g = np.random.default_rng(M + N)
+    C = g.integers(-2_000_000, 2_000_000, size=(M, N), dtype=np.int32)
+    SCA = g.uniform(0.5, 8, size=M).astype(np.float32)
+    SCB = g.uniform(0.01, 0.2, size=N).astype(np.float32)
+    b = (g.standard_normal(N) * 0.01).astype(np.float16) if bias else None
+    out = i8.i8_int8_mm_dequant(dev(C), dev(SCA), dev(SCB), None if b is None else dev(b))
+    assert_close(host(out), oracle.int8_mm_dequant(C, SCA, SCB, b), "mm_dequant")
+
+
+@pytest.mark.parametrize("N,K", [(3, 16), (520, 1040), (4096, 4096)])
+def test_dequant(i8, N, K):
+    W = wl.weight(N + K, N, K)
+    CB, SCB = oracle.quantize_weight_rowwise(W)
+    Wg = i8.i8_dequant(dev(CB), dev(SCB))
+    assert_close(host(Wg), oracle.dequant(CB, SCB), "dequant")
+
+
+# ------------------------------------------------------------------ fused forward
+def _forward_case(i8, M, N, K, n_out, tau, with_bias, cap=256, mag=(20.0, 60.0), seed=0):
+    X, _ = act(M, K, n_out, mag, seed=seed + M + N + K)
+    W = wl.weight(seed + 5, N, K)
+    b = wl.bias(seed + 6, N) if with_bias else None
+    CB, SCB, _ = i8.i8_quantize_rowwise(dev(W), 0.0)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    assert np.array_equal(host(CB), rCB)
+    out, ws = i8.i8_linear8bit_forward(dev(X), CB, SCB, None if b is None else dev(b), tau,
+                                       max_outlier_cols=cap)
+    code, count = i8.i8_read_status(ws)
+    ref = oracle.linear8bit_forward(X, rCB, rSCB, b, tau)
+    _, _, rcols = oracle.quantize_rowwise(X, tau)
+    return host(out), ref, code, count, len(rcols)
+
+
+FSHAPES = [
+    (16, 1024, 1024, 2, 6.0, True),      # the single-linear workload
+    (1, 16, 16, 0, 6.0, False),
+    (37, 300, 272, 3, 6.0, True),
+    (130, 520, 1040, 5, 6.0, False),
+    (256, 512, 4096, 4, 6.0, True),
+    (300, 257, 160, 0, 0.0, True),
+    (513, 700, 2048, 70, 6.0, True),     # two fp16 k-blocks of outliers
+    (200, 384, 512, 3, 0.0, False),      # threshold 0: outlier columns stay on the int8 path
+    (4, 28672, 8192, 8, 6.0, False),     # decode-shaped
+]
+
+
+@pytest.mark.parametrize("M,N,K,n_out,tau,with_bias", FSHAPES)
+def test_linear8bit_forward(i8, M, N, K, n_out, tau, with_bias):
+    out, ref, code, count, n_ref = _forward_case(i8, M, N, K, n_out, tau, with_bias)
+    assert code == 0
+    assert count == (n_ref if tau > 0 else 0)
+    assert_close(out, ref, "forward")
+
+
+def test_forward_all_columns_outliers(i8):
+    """Threshold below every magnitude: the int8 path is empty and out is the fp16 path alone."""
+    M, N, K = 64, 256, 128
+    X, _ = act(M, K, 0, seed=3)
+    X[0] = np.where(np.abs(X[0]) < 1e-2, np.float16(0.5), X[0])
+    out, ref, code, count, n_ref = None, None, None, None, None
+    W = wl.weight(8, N, K)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    o, ws = i8.i8_linear8bit_forward(dev(X), dev(rCB), dev(rSCB), None, 1e-3, max_outlier_cols=K)
+    code, count = i8.i8_read_status(ws)
+    assert code == 0 and count == K
+    assert_close(host(o), oracle.linear8bit_forward(X, rCB, rSCB, None, 1e-3), "all-outlier")
+
+
+def test_forward_outlier_overflow_status(i8):
+    M, N, K = 32, 256, 512
+    X, _ = act(M, K, 20, seed=4)
+    W = wl.weight(9, N, K)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    _, ws = i8.i8_linear8bit_forward(dev(X), dev(rCB), dev(rSCB), None, 6.0, max_outlier_cols=8)
+    code, count = i8.i8_read_status(ws)
+    assert code == 6 and count == 20
+    # the same workspace recovers on the next call with enough capacity
+    o, ws = i8.i8_linear8bit_forward(dev(X), dev(rCB), dev(rSCB), None, 6.0, max_outlier_cols=64)
+    assert i8.i8_read_status(ws) == (0, 20)
+    assert_close(host(o), oracle.linear8bit_forward(X, rCB, rSCB, None, 6.0), "after overflow")
+
+
+def test_forward_deterministic(i8):
+    X, _ = act(300, 1024, 3, seed=5)
+    W = wl.weight(10, 777, 1024)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    dX, dCB, dSCB = dev(X), dev(rCB), dev(rSCB)
+    a, ws = i8.i8_linear8bit_forward(dX, dCB, dSCB, None, 6.0)
+    b, _ = i8.i8_linear8bit_forward(dX, dCB, dSCB, None, 6.0, workspace=ws)
+    assert torch.equal(a, b)
+
+
+def test_opt_mlp_pair_chain(i8):
+    """OPT-350m-shaped fc1 -> ReLU -> fc2, each side chained on its own results."""
+    W = wl.workloads()["C2"]
+    l1, l2 = W.layers
+    X, _, W1, b1 = wl.layer_inputs(2, 0, l1)
+    _, _, W2, b2 = wl.layer_inputs(2, 1, l2)
+    rCB1, rSCB1 = oracle.quantize_weight_rowwise(W1)
+    rCB2, rSCB2 = oracle.quantize_weight_rowwise(W2)
+    h = oracle.linear8bit_forward(X, rCB1, rSCB1, b1, 6.0)
+    h = np.maximum(h, np.float16(0))
+    ref2 = oracle.linear8bit_forward(h, rCB2, rSCB2, b2, 6.0)
+    CB1, SCB1, _ = i8.i8_quantize_rowwise(dev(W1), 0.0)
+    CB2, SCB2, _ = i8.i8_quantize_rowwise(dev(W2), 0.0)
+    o1, _ = i8.i8_linear8bit_forward(dev(X), CB1, SCB1, dev(b1), 6.0)
+    assert_close(host(o1), oracle.linear8bit_forward(X, rCB1, rSCB1, b1, 6.0), "fc1")
+    o2, _ = i8.i8_linear8bit_forward(torch.relu(o1).contiguous(), CB2, SCB2, dev(b2), 6.0)
+    assert_close(host(o2), ref2, "fc2 chained")
+    # fc2 on the oracle's own hidden state: codes are then bit-exact
+    CA2, SCA2, _ = i8.i8_quantize_rowwise(dev(h), 6.0)
+    rCA2, rSCA2, _ = oracle.quantize_rowwise(h, 6.0)
+    assert np.array_equal(host(CA2), rCA2)
+    o2b, _ = i8.i8_linear8bit_forward(dev(h), CB2, SCB2, dev(b2), 6.0)
+    assert_close(host(o2b), ref2, "fc2 on oracle hidden")
+
+
+def test_selftest_bounded_wait_times_out(i8):
+    import time
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    i8.i8_selftest_bounded_wait(st, 50_000_000)   # 50 ms
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 10
+    assert int(st.item()) == 5   # I8_ERR_TIMEOUT, and the context is still usable:
+    assert torch.ones(4, device="cuda").sum().item() == 4
