@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the LLM.int8() Linear8bitLt forward hot path on B200.
+
+One step = one forward pass of every linear of the workload (default: the seven
+linears of a Llama-7B-shaped decoder layer at 4096 prefill tokens), each
+linear = fused quantise + outlier prepare + tcgen05 int8 GEMM with the fused
+dequant / bias / fp16-outlier epilogue.  Inputs are resident in HBM when the
+timed region starts; weights are quantised once before it (load time).
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on a
+bounded row sample of the same workload instead (the slow reference arm).
+
+Multi-GPU: the path has no exchange step, so ``--gpus N`` under torchrun runs N
+independent replicas (weak scaling, no data-path collective); the timed region
+is bracketed by barriers and the slowest rank's device time is reported.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int8_mixed_precision_vectorwise_b200 import workloads as wl  # noqa: E402
+
+METRIC = "LLM.int8() linear TOPS (2MNK/s) vs int8 TC peak; decode weight-read GB/s"
+MAX_OUTLIER_COLS = 256
+GEMM_SOURCES = ("int8_mixed_precision_vectorwise_b200/csrc/gemm_tcgen05.cu",
+                "int8_mixed_precision_vectorwise_b200/csrc/ptx.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_tcgen05_llama7b_prefill_traffic.txt")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="C3")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="rows per linear in the CPU oracle sample")
+    return ap.parse_args()
+
+
+def describe(W: wl.Workload) -> str:
+    parts = [f"{L.name} {L.M}x{L.K}->{L.N}" + (f" ({L.n_out} outlier cols U{L.mag})" if L.n_out else "")
+             for L in W.layers]
+    return f"{W.key}: " + "; ".join(parts) + f"; threshold {W.layers[0].threshold:g}"
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic():
+    """Per-launch DRAM bytes of the GEMM from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    try:
+        kv = dict(l.strip().split("=", 1) for l in open(TRAFFIC_FILE) if "=" in l and not l.startswith("#"))
+        if kv.get("kernel_sha") == gemm_source_sha():
+            return float(kv["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": getattr(self, "err", "no NVML")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        mask = 0
+        for _, r in self.samples:
+            mask |= int(r)
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if mask & b], "samples": len(mhz),
+                "sm_mhz_min": min(mhz)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def cpu_oracle_steps(layers_np, rows: int, steps: int, min_seconds: float = 0.0):
+    """Run the oracle forward on the first `rows` rows of every linear; returns (seconds per step, ops per step)."""
+    import oracle
+    ops = sum(2 * min(rows, X.shape[0]) * CB.shape[0] * X.shape[1] for X, CB, _, _, _ in layers_np)
+    times = []
+    t_all = time.perf_counter()
+    k = 0
+    while k < steps or (time.perf_counter() - t_all) < min_seconds:
+        t0 = time.perf_counter()
+        for X, CB, SCB, b, tau in layers_np:
+            oracle.linear8bit_forward(X[:rows], CB, SCB, b, tau)
+        times.append(time.perf_counter() - t0)
+        k += 1
+    return times, ops
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:  # noqa: BLE001
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_layers(W: wl.Workload, seed: int):
+    import oracle
+    out = []
+    for li, L in enumerate(W.layers):
+        X, _, Wt, b = wl.layer_inputs(seed, li, L)
+        if X is None:   # chained input: the oracle feeds itself (ReLU of its own previous output)
+            pX, pCB, pSCB, pb, ptau = out[-1]
+            X = np.maximum(oracle.linear8bit_forward(pX, pCB, pSCB, pb, ptau), np.float16(0))
+        CB, SCB = oracle.quantize_weight_rowwise(Wt)
+        out.append((X, CB, SCB, b, L.threshold))
+    return out
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    W = wl.workloads()[args.workload]
+    layers_np = oracle_layers(W, wl.seed_of(args.workload))
+    rows = args.cpu_rows
+    cpu_oracle_steps(layers_np, rows, max(args.warmup, 0))
+    times, ops = cpu_oracle_steps(layers_np, rows, args.steps)
+    t = sum(times)
+    value = ops * args.steps / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": describe(W), "sample_rows_per_linear": rows, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"first {rows} rows of every linear of the workload per step "
+                                   "(oracle quantises the sample, exact int product, float64 dequant)"},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import int8_mixed_precision_vectorwise_b200 as i8
+    from int8_mixed_precision_vectorwise_b200 import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device: the library has no CPU path")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    i8.lib()
+
+    W = wl.workloads()[args.workload]
+    seed = wl.seed_of(args.workload)
+    st = torch.cuda.current_stream(dev)
+
+    # ---- inputs (seeded host arrays -> HBM), weight prep on the GPU (load time)
+    layers = []
+    for li, L in enumerate(W.layers):
+        X, _, Wt, b = wl.layer_inputs(seed, li, L)
+        dW = torch.from_numpy(Wt).to(dev)
+        CB, SCB, _ = i8.i8_quantize_rowwise(dW, 0.0)
+        del dW
+        dX = torch.from_numpy(X).to(dev) if X is not None else None
+        db = torch.from_numpy(b).to(dev) if b is not None else None
+        out = torch.empty((L.M, L.N), dtype=torch.float16, device=dev)
+        ws = torch.empty((i8.i8_linear8bit_workspace_size(L.M, L.N, L.K, MAX_OUTLIER_COLS),),
+                         dtype=torch.uint8, device=dev)
+        layers.append(dict(L=L, X=dX, CB=CB, SCB=SCB, b=db, out=out, ws=ws, X_host=X))
+    for li, d in enumerate(layers):      # chained inputs read the previous layer's output buffer
+        if d["X"] is None:
+            d["X"] = layers[li - 1]["out"]
+            d["chained"] = True
+    ops_per_step = sum(d["L"].ops for d in layers)
+    n_launch_per_step = sum(2 + (1 if d["L"].threshold > 0 else 0) for d in layers)
+
+    def step(gemm_events=None):
+        for li, d in enumerate(layers):
+            L = d["L"]
+            i8.i8_linear8bit_prepare(d["X"], d["CB"], L.threshold, d["ws"], MAX_OUTLIER_COLS)
+            if gemm_events is not None:
+                gemm_events[li][0].record(st)
+            i8.i8_linear8bit_matmul_dequant(d["CB"], d["SCB"], d["b"], L.M, L.threshold, d["out"], d["ws"],
+                                            MAX_OUTLIER_COLS)
+            if gemm_events is not None:
+                gemm_events[li][1].record(st)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    for d in layers:
+        code, _ = i8.i8_read_status(d["ws"])
+        if code != 0:
+            raise RuntimeError(f"device status {i8.STATUS.get(code, code)} on {d['L'].name}")
+
+    K = args.steps
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in layers]
+          for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    barrier()
+    with sampler:
+        e0.record(st)
+        for k in range(K):
+            step(ev[k])
+        e1.record(st)
+        barrier()
+    ms = e0.elapsed_time(e1)
+    gemm_ms = sum(a.elapsed_time(b) for row in ev for a, b in row)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end: host inputs -> device -> forward -> host outputs, per step
+    e2e = None
+    if not args.no_e2e:
+        h_in = []
+        for d in layers:
+            h_in.append(None if d.get("chained") else torch.from_numpy(d["X_host"]).pin_memory())
+        h_out = [torch.empty(d["out"].shape, dtype=torch.float16).pin_memory() for d in layers]
+        Ke = min(K, 20)
+
+        def e2e_step():
+            for li, d in enumerate(layers):
+                L = d["L"]
+                if h_in[li] is not None:
+                    d["X"].copy_(h_in[li], non_blocking=True)
+                i8.i8_linear8bit_forward(d["X"], d["CB"], d["SCB"], d["b"], L.threshold, out=d["out"],
+                                         workspace=d["ws"], max_outlier_cols=MAX_OUTLIER_COLS)
+                h_out[li].copy_(d["out"], non_blocking=True)
+        e2e_step()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(st)
+        for _ in range(Ke):
+            e2e_step()
+        f1.record(st)
+        barrier()
+        te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(h.numel() * 2 for h in h_in if h is not None)
+        d2h = sum(h.numel() * 2 for h in h_out)
+        e2e = {"value": world * ops_per_step * Ke / (float(te.item()) / 1e3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
+               "ms_per_step": float(te.item()) / Ke}
+
+    for d in layers:
+        code, _ = i8.i8_read_status(d["ws"])
+        if code != 0:
+            raise RuntimeError(f"device status {i8.STATUS.get(code, code)} on {d['L'].name}")
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        layers_np = oracle_layers(W, seed)
+        times, cops = cpu_oracle_steps(layers_np, args.cpu_rows, 3, min_seconds=10.0)
+        cpu = {"value": cops * len(times) / sum(times) / 1e12, "unit": "TOPS", "cores": cpu_threads(),
+               "kind": "oracle",
+               "sample": f"first {args.cpu_rows} rows of each of the {len(layers_np)} linears, "
+                         f"{len(times)} passes ({sum(times):.1f} s)"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = measured_peaks()
+    if peaks:
+        peak = 2.0 * float(peaks["bf16_tflops_sustained"])
+        peak_src = "of measured: int8 = 2 x bf16_tflops_sustained (nominal int8:bf16 = 4.5:2.25)"
+    else:
+        peak = 2.0 * 1400.0
+        peak_src = "of fallback: int8 = 2 x 1.4 PFLOP/s sustained bf16"
+    gemm_launches = K * len(layers)
+    achieved = ops_per_step * K / (gemm_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": world * ops_per_step * K / (ms_max / 1e3) / 1e12,
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_max / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": describe(W), "tokens": W.layers[0].M, "linears": len(layers),
+                   "max_outlier_cols": MAX_OUTLIER_COLS,
+                   "l2": "per-step working set > 126 MB L2 (int8 weights alone "
+                         f"{sum(d['L'].N * d['L'].K for d in layers) / 1e6:.0f} MB); no flush",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_i8_tcgen05", "achieved": achieved, "peak": peak,
+                     "unit": "TOPS", "frac": achieved / peak, "traffic": read_traffic(),
+                     "peak_source": peak_src, "gemm_ms_per_step": gemm_ms / K,
+                     "gemm_share_of_step": gemm_ms / ms},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": sampler.summary(),
+        "gpu_launches": K * n_launch_per_step,
+        "gpu_launches_note": f"per step per linear: quantise + outlier prepare + GEMM ({gemm_launches} GEMMs)",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -150,14 +150,33 @@ I8_API size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_
  *   workspace / workspace_bytes: see i8_linear8bit_workspace_size.
  *   max_outlier_cols: capacity for |O|; if more columns reach the threshold,
  *   the status word becomes I8_ERR_OUTLIER_OVERFLOW and out is unspecified.
- * Enqueues a small memset plus four kernels (quantise, outlier prepare,
- * tensor-core GEMM with fused dequant epilogue; a split-K reduction kernel is
- * used for M <= 16).
+ * Enqueues one small memset and three kernels: the fused quantiser, the
+ * outlier preparation (skipped when threshold == 0) and the tensor-core GEMM
+ * with the dequant epilogue.  Identical to i8_linear8bit_prepare followed by
+ * i8_linear8bit_matmul_dequant on the same stream and workspace.
  */
 I8_API i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const float* SCB,
                                 const i8_half* bias, int M, int N, int K, float threshold,
                                 i8_half* out, void* workspace, size_t workspace_bytes,
                                 int max_outlier_cols, i8_stream_t stream);
+
+/*
+ * The two halves of i8_linear8bit_forward, for callers that want to place
+ * work or events between them (same arguments, same workspace, same stream):
+ *   i8_linear8bit_prepare: clears the status word and bitmap, quantises X into
+ *     the workspace (CA, SCA, outlier bitmap) and, when threshold > 0, builds
+ *     the outlier column list, zeroes CA's outlier columns and gathers the fp16
+ *     operands X[:, O] and CB[:, O].
+ *   i8_linear8bit_matmul_dequant: the tensor-core GEMM with the fused
+ *     dequant / bias / outlier epilogue, reading the prepared workspace.
+ */
+I8_API i8_status i8_linear8bit_prepare(const i8_half* X, const int8_t* CB, int M, int N, int K,
+                                       float threshold, void* workspace, size_t workspace_bytes,
+                                       int max_outlier_cols, i8_stream_t stream);
+I8_API i8_status i8_linear8bit_matmul_dequant(const int8_t* CB, const float* SCB, const i8_half* bias,
+                                              int M, int N, int K, float threshold, i8_half* out,
+                                              void* workspace, size_t workspace_bytes,
+                                              int max_outlier_cols, i8_stream_t stream);
 
 /*
  * i8_read_status — synchronise `stream` and return the device status word of

@@ -13,6 +13,8 @@ from ._binding import (  # noqa: F401
     i8_int8_linear_matmul,
     i8_int8_mm_dequant,
     i8_linear8bit_forward,
+    i8_linear8bit_matmul_dequant,
+    i8_linear8bit_prepare,
     i8_linear8bit_workspace_size,
     i8_outlier_columns,
     i8_quantize_rowwise,

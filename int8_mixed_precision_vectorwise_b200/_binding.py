@@ -31,7 +31,7 @@ I8_OK = 0
 EXPORTS = (
     "i8_status_string", "i8_quantize_rowwise", "i8_outlier_columns", "i8_int8_linear_matmul",
     "i8_int8_mm_dequant", "i8_dequant", "i8_linear8bit_workspace_size", "i8_linear8bit_forward",
-    "i8_read_status", "i8_selftest_bounded_wait",
+    "i8_read_status", "i8_selftest_bounded_wait", "i8_linear8bit_prepare", "i8_linear8bit_matmul_dequant",
 )
 
 
@@ -60,6 +60,8 @@ def _declare(lib):
         "i8_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
         "i8_linear8bit_workspace_size": (_S, [_I, _I, _I, _I]),
         "i8_linear8bit_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
+        "i8_linear8bit_prepare": (_I, [_P, _P, _I, _I, _I, _F, _P, _S, _I, _P]),
+        "i8_linear8bit_matmul_dequant": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
         "i8_read_status": (_I, [_P, _P, _P]),
         "i8_selftest_bounded_wait": (_I, [_P, ctypes.c_uint64, _P]),
     }
@@ -202,6 +204,28 @@ def i8_linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, out=Non
         _ptr(X), _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out),
         _ptr(workspace), workspace.numel(), max_outlier_cols, _stream(dev)))
     return out, workspace
+
+
+def i8_linear8bit_prepare(X, CB, threshold: float, workspace, max_outlier_cols: int = 256):
+    """First half of the forward: quantise X and prepare the outlier operands in `workspace`."""
+    _need(X, torch.float16, "X", 2)
+    _need(CB, torch.int8, "CB", 2)
+    M, K = X.shape
+    N = CB.shape[0]
+    _check("i8_linear8bit_prepare", lib().i8_linear8bit_prepare(
+        _ptr(X), _ptr(CB), M, N, K, float(threshold), _ptr(workspace), workspace.numel(),
+        max_outlier_cols, _stream(X.device)))
+
+
+def i8_linear8bit_matmul_dequant(CB, SCB, bias, M: int, threshold: float, out, workspace,
+                                 max_outlier_cols: int = 256):
+    """Second half of the forward: the tensor-core GEMM with the fused epilogue."""
+    _need(CB, torch.int8, "CB", 2)
+    N, K = CB.shape
+    _check("i8_linear8bit_matmul_dequant", lib().i8_linear8bit_matmul_dequant(
+        _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out), _ptr(workspace),
+        workspace.numel(), max_outlier_cols, _stream(CB.device)))
+    return out
 
 
 def i8_read_status(workspace):

@@ -134,6 +134,81 @@ i8_status run_gemm(const int8_t* A, const int8_t* B, int M, int N, int K, const 
 
 }  // namespace
 
+namespace {
+
+// Validation shared by the forward and its two stages; fills the layout.
+i8_status check_forward(const i8_half* X, const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N,
+                        int K, float threshold, const i8_half* out, bool need_out, const void* workspace,
+                        size_t workspace_bytes, int max_outlier_cols, WsLayout* L) {
+  if (!X || !workspace || (need_out && (!out || !SCB))) return I8_ERR_INVALID_ARG;
+  i8_status s = check_gemm_operands(X, CB, M, N, K);
+  if (s != I8_OK) return s;
+  if (check_threshold(threshold) != I8_OK || max_outlier_cols < 0) return I8_ERR_INVALID_ARG;
+  if (max_outlier_cols > kMaxOutlierCap) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (need_out && (!aligned16(out) || (bias && !aligned16(bias)))) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!ws_layout(M, N, K, max_outlier_cols, L)) return I8_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < L->total) return I8_ERR_WORKSPACE;
+  return I8_OK;
+}
+
+struct WsPtrs {
+  uint32_t* hdr;
+  uint32_t* bitmap;
+  int32_t* idx;
+  float* SCA;
+  int8_t* CA;
+  __half* XO;
+  __half* WO;
+};
+
+WsPtrs ws_ptrs(void* workspace, const WsLayout& L) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return WsPtrs{reinterpret_cast<uint32_t*>(ws + L.hdr), reinterpret_cast<uint32_t*>(ws + L.bitmap),
+                reinterpret_cast<int32_t*>(ws + L.idx),  reinterpret_cast<float*>(ws + L.sca),
+                reinterpret_cast<int8_t*>(ws + L.ca),    reinterpret_cast<__half*>(ws + L.xo),
+                reinterpret_cast<__half*>(ws + L.wo)};
+}
+
+i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int K, float threshold, void* workspace,
+                          int cap, const WsLayout& L, cudaStream_t st) {
+  const WsPtrs w = ws_ptrs(workspace, L);
+  const __half* Xh = reinterpret_cast<const __half*>(X);
+  const bool outliers = threshold > 0.f;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  // status word, counts and the bitmap are contiguous: one memset clears them
+  if (cudaMemsetAsync(workspace, 0, L.bitmap + static_cast<size_t>((K + 31) / 32) * 4, st) != cudaSuccess)
+    return I8_ERR_CUDA;
+  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr, st));
+  if (s != I8_OK || !outliers) return s;
+  return cuda_status(i8lt::launch_outlier_prepare(w.bitmap, K, cap, reinterpret_cast<int32_t*>(w.hdr + 2),
+                                                  reinterpret_cast<int32_t*>(w.hdr + 1), w.idx, w.hdr, w.CA, Xh, M,
+                                                  cap > 0 ? w.XO : nullptr, CB, N, cap > 0 ? w.WO : nullptr, L.ld_o,
+                                                  sms, st));
+}
+
+i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N, int K,
+                                 float threshold, i8_half* out, void* workspace, int cap, const WsLayout& L,
+                                 cudaStream_t st) {
+  const WsPtrs w = ws_ptrs(workspace, L);
+  const bool with_o = threshold > 0.f && cap > 0;
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.SCA = w.SCA;
+  a.SCB = SCB;
+  a.bias = reinterpret_cast<const __half*>(bias);
+  a.out = reinterpret_cast<__half*>(out);
+  a.n_used = with_o ? reinterpret_cast<const int32_t*>(w.hdr + 1) : nullptr;
+  a.out_cap = cap;
+  a.status = w.hdr;
+  a.wait_limit_ns = kWaitLimitNs;
+  return run_gemm(w.CA, CB, M, N, K, a, false, with_o ? w.XO : nullptr, with_o ? w.WO : nullptr, L.ld_o, st);
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* i8_status_string(i8_status s) {
@@ -226,61 +301,40 @@ size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_cols) {
   return L.total;
 }
 
+
+i8_status i8_linear8bit_prepare(const i8_half* X, const int8_t* CB, int M, int N, int K, float threshold,
+                                void* workspace, size_t workspace_bytes, int max_outlier_cols, i8_stream_t stream) {
+  WsLayout L;
+  i8_status s = check_forward(X, CB, nullptr, nullptr, M, N, K, threshold, nullptr, false, workspace,
+                              workspace_bytes, max_outlier_cols, &L);
+  if (s != I8_OK) return s;
+  return enqueue_prepare(X, CB, M, N, K, threshold, workspace, max_outlier_cols, L,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+i8_status i8_linear8bit_matmul_dequant(const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N, int K,
+                                       float threshold, i8_half* out, void* workspace, size_t workspace_bytes,
+                                       int max_outlier_cols, i8_stream_t stream) {
+  WsLayout L;
+  // X is not read by this stage; CB stands in for it in the shared pointer checks.
+  i8_status s = check_forward(reinterpret_cast<const i8_half*>(CB), CB, SCB, bias, M, N, K, threshold, out, true,
+                              workspace, workspace_bytes, max_outlier_cols, &L);
+  if (s != I8_OK) return s;
+  return enqueue_matmul_dequant(CB, SCB, bias, M, N, K, threshold, out, workspace, max_outlier_cols, L,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
 i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const float* SCB, const i8_half* bias, int M,
                                 int N, int K, float threshold, i8_half* out, void* workspace,
                                 size_t workspace_bytes, int max_outlier_cols, i8_stream_t stream) {
-  if (!X || !out || !workspace) return I8_ERR_INVALID_ARG;
-  i8_status s = check_gemm_operands(X, CB, M, N, K);
-  if (s != I8_OK) return s;
-  if (!SCB) return I8_ERR_INVALID_ARG;
-  if (check_threshold(threshold) != I8_OK || max_outlier_cols < 0) return I8_ERR_INVALID_ARG;
-  if (max_outlier_cols > kMaxOutlierCap) return I8_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(out) || (bias && !aligned16(bias))) return I8_ERR_UNSUPPORTED_SHAPE;
   WsLayout L;
-  if (!ws_layout(M, N, K, max_outlier_cols, &L)) return I8_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < L.total) return I8_ERR_WORKSPACE;
-
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* hdr = reinterpret_cast<uint32_t*>(ws + L.hdr);
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ws + L.bitmap);
-  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
-  float* SCA = reinterpret_cast<float*>(ws + L.sca);
-  int8_t* CA = reinterpret_cast<int8_t*>(ws + L.ca);
-  __half* XO = reinterpret_cast<__half*>(ws + L.xo);
-  __half* WO = reinterpret_cast<__half*>(ws + L.wo);
-  const __half* Xh = reinterpret_cast<const __half*>(X);
-  const bool outliers = threshold > 0.f;
-
-  const int sms = num_sms();
-  if (sms <= 0) return I8_ERR_CUDA;
-  // status word, counts and the bitmap are contiguous: one memset clears them
-  if (cudaMemsetAsync(ws, 0, L.bitmap + static_cast<size_t>((K + 31) / 32) * 4, st) != cudaSuccess)
-    return I8_ERR_CUDA;
-  s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, outliers ? bitmap : nullptr, st));
+  i8_status s = check_forward(X, CB, SCB, bias, M, N, K, threshold, out, true, workspace, workspace_bytes,
+                              max_outlier_cols, &L);
   if (s != I8_OK) return s;
-  if (outliers) {
-    const int cap = max_outlier_cols;
-    s = cuda_status(i8lt::launch_outlier_prepare(bitmap, K, cap, reinterpret_cast<int32_t*>(hdr + 2),
-                                                 reinterpret_cast<int32_t*>(hdr + 1), idx, hdr, CA, Xh, M,
-                                                 cap > 0 ? XO : nullptr, CB, N, cap > 0 ? WO : nullptr, L.ld_o,
-                                                 sms, st));
-    if (s != I8_OK) return s;
-  }
-  GemmArgs a{};
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.SCA = SCA;
-  a.SCB = SCB;
-  a.bias = reinterpret_cast<const __half*>(bias);
-  a.out = reinterpret_cast<__half*>(out);
-  a.n_used = (outliers && max_outlier_cols > 0) ? reinterpret_cast<const int32_t*>(hdr + 1) : nullptr;
-  a.out_cap = max_outlier_cols;
-  a.status = hdr;
-  a.wait_limit_ns = kWaitLimitNs;
-  const bool with_o = outliers && max_outlier_cols > 0;
-  return run_gemm(CA, CB, M, N, K, a, false, with_o ? XO : nullptr, with_o ? WO : nullptr, L.ld_o, st);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = enqueue_prepare(X, CB, M, N, K, threshold, workspace, max_outlier_cols, L, st);
+  if (s != I8_OK) return s;
+  return enqueue_matmul_dequant(CB, SCB, bias, M, N, K, threshold, out, workspace, max_outlier_cols, L, st);
 }
 
 i8_status i8_read_status(const void* workspace, int32_t* count, i8_stream_t stream) {
