@@ -188,6 +188,36 @@ I8_API i8_status i8_linear8bit_matmul_dequant(const int8_t* CB, const float* SCB
 I8_API i8_status i8_read_status(const void* workspace, int32_t* count, i8_stream_t stream);
 
 /*
+ * i8_linear8bit_forward_static — the same forward as i8_linear8bit_forward,
+ * for callers that cannot hand the library a workspace.  The pages have no
+ * counterpart to this entry point.
+ *
+ * Some callers cannot allocate device memory where they run the forward:
+ * plugin and inference-server hooks that are handed a stream but no allocator
+ * or workspace, code inside a framework whose own caching allocator owns the
+ * device memory, and latency-critical loops that must not call cudaMalloc
+ * (it can synchronise the whole device) or take an allocator's locks.  This
+ * entry point allocates nothing: its scratch is a
+ * fixed 32 MiB device array built into the library (each GPU that loads the
+ * library keeps it until the process exits).  The caller still passes X, CB,
+ * SCB, bias and out exactly as for i8_linear8bit_forward.
+ *   status_out: optional device pointer to 3 uint32 that receive, in stream
+ *     order, the status word and the used / total outlier-column counts (the
+ *     values i8_read_status reports for a workspace); NULL to skip.
+ * Sizes whose workspace (i8_linear8bit_workspace_size) exceeds 32 MiB are
+ * rejected with I8_ERR_WORKSPACE before anything is enqueued.
+ * The first call on each device looks up the array's device address and must
+ * happen before any stream capture that records this call.  All calls share
+ * the one array and it keeps the previous call's contents (each call clears
+ * what must start at zero), so calls that can overlap on the GPU — on two
+ * streams, or from two host threads — race; serialise them on one stream.
+ */
+I8_API i8_status i8_linear8bit_forward_static(const i8_half* X, const int8_t* CB, const float* SCB,
+                                              const i8_half* bias, int M, int N, int K, float threshold,
+                                              i8_half* out, int max_outlier_cols, uint32_t* status_out,
+                                              i8_stream_t stream);
+
+/*
  * i8_selftest_bounded_wait — failure-detection self test.  Launches one block
  * that waits on a shared-memory barrier that nothing ever completes, with the
  * same bounded-wait routine the GEMM pipeline uses and a limit of

@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     i8_int8_linear_matmul,
     i8_int8_mm_dequant,
     i8_linear8bit_forward,
+    i8_linear8bit_forward_static,
     i8_linear8bit_matmul_dequant,
     i8_linear8bit_prepare,
     i8_linear8bit_workspace_size,

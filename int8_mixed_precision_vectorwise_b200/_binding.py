@@ -32,6 +32,7 @@ EXPORTS = (
     "i8_status_string", "i8_quantize_rowwise", "i8_outlier_columns", "i8_int8_linear_matmul",
     "i8_int8_mm_dequant", "i8_dequant", "i8_linear8bit_workspace_size", "i8_linear8bit_forward",
     "i8_read_status", "i8_selftest_bounded_wait", "i8_linear8bit_prepare", "i8_linear8bit_matmul_dequant",
+    "i8_linear8bit_forward_static",
 )
 
 
@@ -62,6 +63,7 @@ def _declare(lib):
         "i8_linear8bit_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
         "i8_linear8bit_prepare": (_I, [_P, _P, _I, _I, _I, _F, _P, _S, _I, _P]),
         "i8_linear8bit_matmul_dequant": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
+        "i8_linear8bit_forward_static": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P]),
         "i8_read_status": (_I, [_P, _P, _P]),
         "i8_selftest_bounded_wait": (_I, [_P, ctypes.c_uint64, _P]),
     }
@@ -225,6 +227,23 @@ def i8_linear8bit_matmul_dequant(CB, SCB, bias, M: int, threshold: float, out, w
     _check("i8_linear8bit_matmul_dequant", lib().i8_linear8bit_matmul_dequant(
         _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out), _ptr(workspace),
         workspace.numel(), max_outlier_cols, _stream(CB.device)))
+    return out
+
+
+def i8_linear8bit_forward_static(X, CB, SCB, bias=None, threshold: float = 6.0, out=None,
+                                 max_outlier_cols: int = 256, status_out=None):
+    """Forward using the library's built-in scratch instead of a workspace (see include/i8lt.h)."""
+    _need(X, torch.float16, "X", 2)
+    _need(CB, torch.int8, "CB", 2)
+    _need(SCB, torch.float32, "SCB", 1)
+    if bias is not None:
+        _need(bias, torch.float16, "bias", 1)
+    M, K = X.shape
+    N = CB.shape[0]
+    out = torch.empty((M, N), dtype=torch.float16, device=X.device) if out is None else out
+    _check("i8_linear8bit_forward_static", lib().i8_linear8bit_forward_static(
+        _ptr(X), _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out), max_outlier_cols,
+        _ptr(status_out), _stream(X.device)))
     return out
 
 

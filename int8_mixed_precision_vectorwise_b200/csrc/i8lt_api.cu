@@ -209,6 +209,35 @@ i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_ha
 
 }  // namespace
 
+// ---------------------------------------------------------------- allocation-free forward
+// Built-in scratch for i8_linear8bit_forward_static.  It is a plain device
+// array, so every GPU that loads this library holds kStaticScratchBytes of it
+// until the process exits, and every call of that entry point shares it.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+// Device address of g_static_scratch on the current device.  In host code the
+// array's name only stands in for the symbol, so the address is looked up with
+// cudaGetSymbolAddress, once per device, while that device is current.
+i8_status static_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return I8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return I8_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return I8_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* i8_status_string(i8_status s) {
@@ -351,6 +380,32 @@ i8_status i8_selftest_bounded_wait(uint32_t* status, uint64_t limit_ns, i8_strea
   if (!status) return I8_ERR_INVALID_ARG;
   if (limit_ns < 1000000ull || limit_ns > 10000000000ull) return I8_ERR_INVALID_ARG;
   return cuda_status(i8lt::launch_selftest_wait(status, limit_ns, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_linear8bit_forward_static(const i8_half* X, const int8_t* CB, const float* SCB, const i8_half* bias,
+                                       int M, int N, int K, float threshold, i8_half* out, int max_outlier_cols,
+                                       uint32_t* status_out, i8_stream_t stream) {
+  if (!X || !out || !SCB) return I8_ERR_INVALID_ARG;
+  i8_status s = check_gemm_operands(X, CB, M, N, K);
+  if (s != I8_OK) return s;
+  if (check_threshold(threshold) != I8_OK || max_outlier_cols < 0) return I8_ERR_INVALID_ARG;
+  if (max_outlier_cols > kMaxOutlierCap) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(out) || (bias && !aligned16(bias))) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u) != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  WsLayout L;
+  if (!ws_layout(M, N, K, max_outlier_cols, &L)) return I8_ERR_INVALID_ARG;
+  if (L.total > kStaticScratchBytes) return I8_ERR_WORKSPACE;  // needs more than the built-in 32 MiB
+  void* ws = nullptr;
+  s = static_scratch(&ws);
+  if (s != I8_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the prepare stage clears the status word, counts and bitmap; every other
+  // byte it reads back is written earlier in the same call
+  s = enqueue_prepare(X, CB, M, N, K, threshold, ws, max_outlier_cols, L, st);
+  if (s != I8_OK) return s;
+  s = enqueue_matmul_dequant(CB, SCB, bias, M, N, K, threshold, out, ws, max_outlier_cols, L, st);
+  if (s != I8_OK || status_out == nullptr) return s;
+  return cuda_status(cudaMemcpyAsync(status_out, ws, 3 * sizeof(uint32_t), cudaMemcpyDeviceToDevice, st));
 }
 
 }  // extern "C"
