@@ -11,15 +11,24 @@
 // int8_mm_dequant ops of "LLM.int8() Refactoring: Part 1" (section
 // "Deprecations") fused into one kernel.  The raw variant stores C as int32.
 //
-// Block = 6 warps: warp 0 issues TMA loads (one elected lane), warp 1 owns
-// TMEM and issues tcgen05.mma (one lane), warps 2-5 run the epilogue (each
-// warp reads the 32 TMEM lanes of its quadrant).  One CTA per SM walks tiles
-// of 128 x 256 outputs; K is streamed through a 4-stage ring of
-// 128-byte-deep, 128B-swizzled tiles.  The gathered fp16 outlier tiles (64
-// fp16 = 128 bytes deep) reuse the same ring after the int8 k-blocks.
-// TMEM: 512 columns.  Without outliers, two 256-column int32 accumulators
-// alternate between tiles so the epilogue of tile t overlaps the mainloop of
-// tile t+1; with outliers, columns [0,256) hold C and [256,512) hold D.
+// The kernel runs on CTA pairs (clusters of 2, tcgen05 cta_group::2): a pair
+// computes 256 x 256 output tiles; each CTA loads its own 128 rows of A and its
+// own 128 rows of B into its shared memory (plain TMA loads, no multicast) and
+// the leader CTA issues one M=256 MMA over both halves.  Each CTA's TMEM holds
+// the accumulator rows of its half.
+//
+// Block = 10 warps: warp 0 issues TMA loads (one lane), warp 1 owns TMEM and,
+// in the leader, issues tcgen05.mma (one lane); warps 2-9 run the epilogue
+// (two warps per 32-lane TMEM quadrant, one per 128-column half).  K streams
+// through a 6-stage ring of 128-byte-deep, 128B-swizzled tiles; the gathered
+// fp16 outlier tiles (64 fp16 = 128 bytes deep) use the same ring after the
+// int8 k-blocks.  TMEM: 512 columns.  Two 256-column int32 accumulators
+// alternate so the epilogue of tile t overlaps the mainloop of tile t+1.  Up
+// to 16 outlier columns, the epilogue adds the (rank <= 16) outlier product
+// itself with warp-level MMAs (mma.sync m16n8k16) on the gathered operands;
+// with more, tcgen05 kind::f16 MMAs write D into TMEM columns [256,512) and
+// the accumulator is single-buffered.
+// The epilogue writes fp16 32x32 boxes through shared memory with TMA stores.
 #include <cuda_fp16.h>
 
 #include "kernels.cuh"
@@ -29,25 +38,31 @@ namespace i8lt {
 
 namespace {
 
-constexpr int BM = kGemmBM;
-constexpr int BN = kGemmBN;
+constexpr int BM = kGemmBM;          // rows per CTA
+constexpr int BN = kGemmBN;          // columns per pair tile
+constexpr int BNH = BN / 2;          // B rows per CTA
 constexpr int BK = kGemmBKBytes;
-constexpr int STAGES = 4;
-constexpr int EPI_WARPS = 4;
+constexpr int STAGES = 6;
+constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int A_BYTES = BM * BK;
-constexpr int B_BYTES = BN * BK;
+constexpr int B_BYTES = BNH * BK;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+constexpr int OBOX = kGemmOutBox;                // 32 x 32 fp16 output box
+constexpr int STG_BYTES = OBOX * OBOX * 2;       // 2 KB
+constexpr int STG_OFF = RING_BYTES;
+constexpr int STG_TOTAL = EPI_WARPS * 2 * STG_BYTES;
 constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-constexpr int SCALE_OFF = BAR_OFF + ((NUM_BARS * 8 + 15) / 16) * 16;
-constexpr int SCALE_BYTES_PER_WARP = 2 * BN * 4;  // SCB and bias of the current tile, per epilogue warp
-constexpr int MISC_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES_PER_WARP;
+constexpr int BAR_OFF = STG_OFF + STG_TOTAL;
+constexpr int MISC_OFF = BAR_OFF + ((NUM_BARS * 8 + 15) / 16) * 16;
 constexpr int SMEM_USED = MISC_OFF + 16;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack to align the ring to 1024 bytes
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int CHUNKS = BNH / 32;              // 32-column chunks per epilogue warp
+constexpr int SMALL_O = kSmallOutliers;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-static_assert(BN == 256, "accumulator layout assumes 256 columns per tile");
+static_assert(SMALL_O == 16, "the epilogue's warp MMA covers one k-step of 16 outlier columns");
 
 // Wait without an abort flag (used for the final drains, which must really
 // wait for in-flight asynchronous work), still bounded by `limit_ns`.
@@ -64,86 +79,101 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }  // namespace
 
 template <bool RAW>
-__global__ void __launch_bounds__(THREADS, 1)
-    k_gemm_i8_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmXO, const __grid_constant__ CUtensorMap tmWO,
-                      const GemmArgs p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_gemm_i8_tcgen05(const __grid_constant__ GemmMaps tm, const GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);  // used in the leader only
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [2]
-  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2], used in the leader only
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(num_clusters_x());
   const int M = p.M, N = p.N, K = p.K;
-  const int num_m = (M + BM - 1) / BM;
+  const int num_m = (M + 2 * BM - 1) / (2 * BM);
   const int num_n = (N + BN - 1) / BN;
   const int tiles = num_m * num_n;
   const int kb_int = (K + BK - 1) / BK;
   int n_used = 0;
   if (!RAW && p.n_used != nullptr) n_used = min(max(*p.n_used, 0), p.out_cap);
-  const int kb_out = (n_used + 63) / 64;
+  // Few outlier columns are added by the epilogue on CUDA cores (a rank-n
+  // update) so the TMEM accumulators stay double-buffered; more go through an
+  // fp16 MMA into a second accumulator.
+  const bool small_o = n_used > 0 && n_used <= SMALL_O && p.XO != nullptr && p.WO != nullptr;
+  const int kb_out = small_o ? 0 : (n_used + 63) / 64;
   const int kb_all = kb_int + kb_out;
   const bool dbl = kb_out == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1);   // the leader's expect-tx arrival; the bytes of both CTAs complete it
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 32 * EPI_WARPS);
+      mbar_init(&acc_empty[b], 2 * EPI_WARPS);
     }
     mbar_init(mma_done, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tm.A);
+    tma_prefetch_desc(&tm.B);
     if (kb_out > 0) {
-      tma_prefetch_desc(&tmXO);
-      tma_prefetch_desc(&tmWO);
+      tma_prefetch_desc(&tm.XO);
+      tma_prefetch_desc(&tm.WO);
     }
+    if (!RAW && p.tma_store) tma_prefetch_desc(&tm.Out);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(s_tmem, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before_sync();
-  __syncthreads();
+  cluster_sync();  // barriers initialised and TMEM allocated in both CTAs of the pair
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
     if (lane == 0) {
+      const uint32_t full0_leader = map_to_rank(smem_addr(&full[0]), 0);
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t filled = 0, fill_parity = 0;  // per stage: ever filled / full-barrier parity of the last fill
-      for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x) {
-        const int m0 = (tile % num_m) * BM;
-        const int n0 = (tile / num_m) * BN;
+      uint32_t filled = 0, fill_parity = 0;  // leader: per stage, ever filled / parity of the last fill
+      for (int tile = pair; tile < tiles && !*s_abort; tile += npairs) {
+        const int m0 = (tile % num_m) * (2 * BM) + static_cast<int>(rank) * BM;
+        const int nb0 = (tile / num_m) * BN + static_cast<int>(rank) * BNH;
         for (int kb = 0; kb < kb_all; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.status, p.wait_limit_ns)) break;
           uint8_t* sa = smem + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          filled |= 1u << stage;
-          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          const uint32_t bar = full0_leader + static_cast<uint32_t>(stage) * 8u;
+          if (leader) {
+            // one arrival that expects the bytes of both CTAs.  The peer's copies
+            // may land first (the transaction count goes negative meanwhile); the
+            // phase cannot complete before this arrival, and the peer cannot
+            // refill the stage before the MMA has consumed it.
+            mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+            filled |= 1u << stage;
+            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          }
           if (kb < kb_int) {
-            tma_load_2d(sa, &tmA, &full[stage], kb * BK, m0);
-            tma_load_2d(sb, &tmB, &full[stage], kb * BK, n0);
+            tma_load_2d_pair(sa, &tm.A, bar, kb * BK, m0);
+            tma_load_2d_pair(sb, &tm.B, bar, kb * BK, nb0);
           } else {
             const int ko = (kb - kb_int) * 64;  // fp16 elements
-            tma_load_2d(sa, &tmXO, &full[stage], ko, m0);
-            tma_load_2d(sb, &tmWO, &full[stage], ko, n0);
+            tma_load_2d_pair(sa, &tm.XO, bar, ko, m0);
+            tma_load_2d_pair(sb, &tm.WO, bar, ko, nb0);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -151,23 +181,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      // Never leave the CTA while a copy may still be landing in shared memory:
-      // every stage this thread filled is either consumed or is waited for here.
+      // Never leave while a copy may still be landing in shared memory.  The
+      // leader's full barriers count both CTAs' bytes; the peer, which cannot
+      // observe them, gives its last copies a bounded grace period.
       if (*s_abort) {
-        for (int s = 0; s < STAGES; ++s)
-          if (filled & (1u << s)) drain_wait(&full[s], (fill_parity >> s) & 1u, p.wait_limit_ns);
+        if (leader) {
+          for (int s = 0; s < STAGES; ++s)
+            if (filled & (1u << s)) drain_wait(&full[s], (fill_parity >> s) & 1u, p.wait_limit_ns);
+        } else {
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_i = idesc_i8_s32(BM, BN);
-      const uint32_t idesc_f = idesc_f16_f32(BM, BN);
+    // ---------------------------------------------------------------- MMA issuer (leader only)
+    if (leader && lane == 0) {
+      const uint32_t idesc_i = idesc_i8_s32(2 * BM, BN);
+      const uint32_t idesc_f = idesc_f16_f32(2 * BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (int tile = blockIdx.x; tile < tiles && !*s_abort; tile += gridDim.x, ++it) {
+      for (int tile = pair; tile < tiles && !*s_abort; tile += npairs, ++it) {
         const int buf = dbl ? (it & 1) : 0;
         const uint32_t use = dbl ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
         if (!mbar_wait_bounded(&acc_empty[buf], (use & 1u) ^ 1u, s_abort, p.status, p.wait_limit_ns)) break;
@@ -187,138 +223,276 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (kb < kb_int) {
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)  // 32 int8 = 32 bytes per MMA
-              mma_i8(d_int, adesc + 2 * k, bdesc + 2 * k, idesc_i, (kb > 0 || k > 0) ? 1u : 0u);
+              mma_i8_pair(d_int, adesc + 2 * k, bdesc + 2 * k, idesc_i, (kb > 0 || k > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)  // 16 fp16 = 32 bytes per MMA
-              mma_f16(d_fp, adesc + 2 * k, bdesc + 2 * k, idesc_f, (kb > kb_int || k > 0) ? 1u : 0u);
+              mma_f16_pair(d_fp, adesc + 2 * k, bdesc + 2 * k, idesc_f, (kb > kb_int || k > 0) ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          tc_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(&acc_full[buf]);
+        tc_commit_pair(&acc_full[buf], 0x3);  // both CTAs' accumulator halves are ready
       }
       // Wait for every MMA this thread issued before TMEM is released.
-      tc_commit(mma_done);
+      tc_commit_pair(mma_done, 0x1);
       drain_wait(mma_done, 0, p.wait_limit_ns);
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- epilogue
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    // Each warp owns 32 accumulator rows (its TMEM lane quadrant) and 128 of
+    // the tile's 256 columns, processed as four 32x32 chunks.  TMEM is read in
+    // the mma.m16n8 accumulator layout (thread t: rows t/4 and t/4+8 of each
+    // 16-row block, columns 2(t%4), 2(t%4)+1 of each 8-column block), so the
+    // few-outlier product can be added with warp MMAs in the same layout.
+    const int ew = warp - 2;                    // 0..7
     const int quad = warp & 3;                  // TMEM lanes this warp may read
+    const int col_half = ew >> 2;               // which 128 of the tile's 256 columns
+    const int g = lane >> 2, tq = lane & 3;     // fragment row / column pair
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const bool vec_ok = RAW ? ((N & 3) == 0) : ((N & 7) == 0);
-    // Each epilogue warp keeps its own copy of the tile's column scales and
-    // bias, so the four warps never wait on one another.
-    float* s_scb = reinterpret_cast<float*>(smem + SCALE_OFF + (warp - 2) * SCALE_BYTES_PER_WARP);
-    float* s_bias = s_scb + BN;
+    const uint32_t acc_empty0_leader = map_to_rank(smem_addr(&acc_empty[0]), 0);
+    uint8_t* stg = smem + STG_OFF + ew * 2 * STG_BYTES;
+    int stg_i = 0;
     int it = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {  // abort is seen by the wait below
-      const int m0 = (tile % num_m) * BM;
-      const int n0 = (tile / num_m) * BN;
-      if (!RAW) {
-        __syncwarp();  // every lane is done with the previous tile's copy
-        for (int c = lane; c < BN; c += 32) {
-          const int n = n0 + c;
-          s_scb[c] = n < N ? p.SCB[n] : 0.f;
-          s_bias[c] = (p.bias != nullptr && n < N) ? __half2float(p.bias[n]) : 0.f;
-        }
-        __syncwarp();
-      }
+    for (int tile = pair; tile < tiles; tile += npairs, ++it) {  // abort is seen by the wait below
+      const int row_base = (tile % num_m) * (2 * BM) + static_cast<int>(rank) * BM + quad * 32;
+      const int n0 = (tile / num_m) * BN + col_half * BNH;
       const int buf = dbl ? (it & 1) : 0;
       const uint32_t use = dbl ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
+      // Everything this tile needs besides the accumulators is fetched before
+      // the accumulator wait, so its latency hides behind the mainloop.
+      // Column scales / bias: lane j holds column cc*32 + j of chunk cc.
+      float sb_r[CHUNKS], bi_r[CHUNKS];
+#pragma unroll
+      for (int cc = 0; cc < CHUNKS; ++cc) {
+        const int n = n0 + cc * 32 + lane;
+        const bool in = !RAW && n < N;
+        sb_r[cc] = in ? __ldg(p.SCB + n) : 0.f;
+        bi_r[cc] = (in && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
+      }
+      // Row scales of this thread's four rows: row_base + g + 8i.
+      float sa4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = row_base + g + 8 * i;
+        sa4[i] = (!RAW && r < M) ? __ldg(p.SCA + r) * (1.0f / 16129.0f) : 0.f;
+      }
+      // Few outliers: A fragments (X[:, O] rows) and B fragments (CB[:, O]
+      // columns of the four chunks) of the 16-wide outlier product.
+      uint32_t af[2][4], bf[CHUNKS][4][2];
+#pragma unroll
+      for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) af[rb][e] = 0u;
+#pragma unroll
+      for (int cc = 0; cc < CHUNKS; ++cc)
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) bf[cc][cb][0] = bf[cc][cb][1] = 0u;
+      if (small_o) {
+#pragma unroll
+        for (int rb = 0; rb < 2; ++rb) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = row_base + rb * 16 + g + 8 * (e & 1);
+            const int k = 2 * tq + 8 * (e >> 1);
+            if (r < M) af[rb][e] = __ldg(reinterpret_cast<const uint32_t*>(p.XO + static_cast<size_t>(r) * p.ld_o + k));
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < CHUNKS; ++cc) {
+#pragma unroll
+          for (int cb = 0; cb < 4; ++cb) {
+            const int n = n0 + cc * 32 + cb * 8 + g;
+            if (n < N) {
+              const uint32_t* w = reinterpret_cast<const uint32_t*>(p.WO + static_cast<size_t>(n) * p.ld_o + 2 * tq);
+              bf[cc][cb][0] = __ldg(w);
+              bf[cc][cb][1] = __ldg(w + 4);
+            }
+          }
+        }
+      }
       // lane 0 waits for the whole warp, so the warp leaves the loop as one
       // (the TMEM loads below are warp-collective)
       int ok = 0;
       if (lane == 0) ok = mbar_wait_bounded(&acc_full[buf], use & 1u, s_abort, p.status, p.wait_limit_ns) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after_sync();
-      const int row = m0 + quad * 32 + lane;
-      const bool row_ok = row < M;
-      const float sa = (!RAW && row_ok) ? p.SCA[row] * (1.0f / 16129.0f) : 0.f;
-      const uint32_t t_int = tmem_base + lane_off + static_cast<uint32_t>(buf * BN);
-      const uint32_t t_fp = tmem_base + lane_off + static_cast<uint32_t>(BN);
-#pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        uint32_t ri[32];
-        tmem_ld_32x32b_x32(t_int + cc * 32, ri);
-        uint32_t rf[32];
-        if (!RAW && kb_out > 0) tmem_ld_32x32b_x32(t_fp + cc * 32, rf);
+      const uint32_t t_int = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + col_half * BNH);
+      const uint32_t t_fp = tmem_base + lane_off + static_cast<uint32_t>(BN + col_half * BNH);
+#pragma unroll
+      for (int cc = 0; cc < CHUNKS; ++cc) {
+        uint32_t c[2][16];  // int32 accumulators of row blocks 0 / 1
+        tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
+        tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
+        uint32_t f[2][16];  // fp32 outlier accumulators (many-outlier path)
+        if (!RAW && kb_out > 0) {
+          tmem_ld_16x256b_x4(t_fp + cc * 32, f[0]);
+          tmem_ld_16x256b_x4(t_fp + (16u << 16) + cc * 32, f[1]);
+        }
         tmem_wait_ld();
         const int nb = n0 + cc * 32;
-        if (!row_ok || nb >= N) continue;
         if (RAW) {
-          int32_t* dst = p.C + static_cast<size_t>(row) * N + nb;
-          if (vec_ok && nb + 32 <= N) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              reinterpret_cast<uint4*>(dst)[q] = make_uint4(ri[4 * q], ri[4 * q + 1], ri[4 * q + 2], ri[4 * q + 3]);
-          } else {
+          for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (nb + j < N) dst[j] = static_cast<int32_t>(ri[j]);
+            for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int r = row_base + rb * 16 + g + 8 * hh;
+                const int n = nb + cb * 8 + 2 * tq;
+                if (r >= M || n >= N) continue;
+                int32_t* dst = p.C + static_cast<size_t>(r) * N + n;
+                const uint32_t v0 = c[rb][4 * cb + 2 * hh], v1 = c[rb][4 * cb + 2 * hh + 1];
+                if ((N & 1) == 0 && n + 1 < N) {
+                  *reinterpret_cast<int2*>(dst) = make_int2(static_cast<int>(v0), static_cast<int>(v1));
+                } else {
+                  dst[0] = static_cast<int32_t>(v0);
+                  if (n + 1 < N) dst[1] = static_cast<int32_t>(v1);
+                }
+              }
+          continue;
+        }
+        // dequant in fragment layout; halves[rb][cb][hh] = (row rb*16+g+8hh, columns cb*8+2tq, +1)
+        uint32_t halves[2][4][2];
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+          const int j = cb * 8 + 2 * tq;
+          const float sb0 = __shfl_sync(0xffffffffu, sb_r[cc], j);
+          const float sb1 = __shfl_sync(0xffffffffu, sb_r[cc], j + 1);
+          const float b0 = __shfl_sync(0xffffffffu, bi_r[cc], j);
+          const float b1 = __shfl_sync(0xffffffffu, bi_r[cc], j + 1);
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            if (small_o) {
+              mma_16x8x16_f16(d, af[rb], bf[cc][cb][0], bf[cc][cb][1]);
+            } else if (kb_out > 0) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) d[e] = __uint_as_float(f[rb][4 * cb + e]);
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const float sa = sa4[2 * rb + hh];
+              const float v0 = fmaf(d[2 * hh], sb0 * (1.0f / 127.0f),
+                                    fmaf(static_cast<float>(static_cast<int32_t>(c[rb][4 * cb + 2 * hh])), sa * sb0, b0));
+              const float v1 = fmaf(d[2 * hh + 1], sb1 * (1.0f / 127.0f),
+                                    fmaf(static_cast<float>(static_cast<int32_t>(c[rb][4 * cb + 2 * hh + 1])), sa * sb1, b1));
+              halves[rb][cb][hh] = pack_half2(v0, v1);
+            }
           }
+        }
+        if (p.tma_store) {
+          // 32 rows x 32 fp16 box through shared memory with the 64-byte
+          // swizzle: 16-byte chunk q of row r sits at chunk q ^ ((r >> 1) & 3)
+          uint8_t* box = stg + stg_i * STG_BYTES;
+          if (lane == 0) tma_store_wait_read<1>();  // the store that last read this buffer is done
+          __syncwarp();
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int r = rb * 16 + g + 8 * hh;
+#pragma unroll
+              for (int cb = 0; cb < 4; ++cb)
+                *reinterpret_cast<uint32_t*>(box + r * 64 + ((cb ^ ((r >> 1) & 3)) << 4) + 4 * tq) =
+                    halves[rb][cb][hh];
+            }
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            if (nb < N && row_base < M) tma_store_2d(&tm.Out, box, nb, row_base);
+            tma_store_commit();
+          }
+          stg_i ^= 1;
         } else {
-          float y[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float sb = s_scb[cc * 32 + j];
-            float v = fmaf(static_cast<float>(static_cast<int32_t>(ri[j])), sa * sb, s_bias[cc * 32 + j]);
-            if (kb_out > 0) v = fmaf(__uint_as_float(rf[j]), sb * (1.0f / 127.0f), v);
-            y[j] = v;
-          }
-          __half* dst = p.out + static_cast<size_t>(row) * N + nb;
-          if (vec_ok && nb + 32 <= N) {
+          for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              reinterpret_cast<uint4*>(dst)[q] =
-                  make_uint4(pack_half2(y[8 * q], y[8 * q + 1]), pack_half2(y[8 * q + 2], y[8 * q + 3]),
-                             pack_half2(y[8 * q + 4], y[8 * q + 5]), pack_half2(y[8 * q + 6], y[8 * q + 7]));
-          } else {
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (nb + j < N) dst[j] = __float2half_rn(y[j]);
-          }
+              for (int cb = 0; cb < 4; ++cb) {
+                const int r = row_base + rb * 16 + g + 8 * hh;
+                const int n = nb + cb * 8 + 2 * tq;
+                if (r >= M || n >= N) continue;
+                __half* dst = p.out + static_cast<size_t>(r) * N + n;
+                const uint32_t hv = halves[rb][cb][hh];
+                if ((N & 1) == 0 && n + 1 < N) {
+                  *reinterpret_cast<uint32_t*>(dst) = hv;
+                } else {
+                  dst[0] = reinterpret_cast<const __half*>(&hv)[0];
+                  if (n + 1 < N) dst[1] = reinterpret_cast<const __half*>(&hv)[1];
+                }
+              }
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(&acc_empty[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0_leader + static_cast<uint32_t>(buf) * 8u);
     }
+    if (!RAW && p.tma_store && lane == 0) tma_store_wait_all<0>();
+    __syncwarp();
   }
 
-  __syncthreads();
+  tc_fence_before_sync();
+  cluster_sync();  // no CTA leaves while its pair may still read its shared memory or signal its barriers
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
-cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmXO,
-                        const CUtensorMap& tmWO, const GemmArgs& a, bool raw_int32, int num_sms, cudaStream_t st) {
-  static bool attr_done[2] = {false, false};
-  const int tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  if (raw_int32) {
-    if (!attr_done[1]) {
-      cudaError_t e = cudaFuncSetAttribute(k_gemm_i8_tcgen05<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           SMEM_ALLOC);
-      if (e != cudaSuccess) return e;
-      attr_done[1] = true;
-    }
-    k_gemm_i8_tcgen05<true><<<grid, THREADS, SMEM_ALLOC, st>>>(tmA, tmB, tmXO, tmWO, a);
-  } else {
-    if (!attr_done[0]) {
-      cudaError_t e = cudaFuncSetAttribute(k_gemm_i8_tcgen05<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           SMEM_ALLOC);
-      if (e != cudaSuccess) return e;
-      attr_done[0] = true;
-    }
-    k_gemm_i8_tcgen05<false><<<grid, THREADS, SMEM_ALLOC, st>>>(tmA, tmB, tmXO, tmWO, a);
+// Number of CTA pairs that fit on the device at once (cached per device).
+static int max_pairs(bool raw, int num_sms) {
+  static int cache[2][64] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int r = raw ? 1 : 0;
+  if (dev >= 0 && dev < 64 && cache[r][dev] > 0) return cache[r][dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1), 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  cudaError_t e = raw ? cudaOccupancyMaxActiveClusters(&n, k_gemm_i8_tcgen05<true>, &cfg)
+                      : cudaOccupancyMaxActiveClusters(&n, k_gemm_i8_tcgen05<false>, &cfg);
+  if (e != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = num_sms / 2;
   }
+  if (dev >= 0 && dev < 64) cache[r][dev] = n;
+  return n;
+}
+
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, bool raw_int32, int num_sms, cudaStream_t st) {
+  static bool attr_done[2] = {false, false};
+  const int raw = raw_int32 ? 1 : 0;
+  if (!attr_done[raw]) {
+    cudaError_t e = raw ? cudaFuncSetAttribute(k_gemm_i8_tcgen05<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               SMEM_ALLOC)
+                        : cudaFuncSetAttribute(k_gemm_i8_tcgen05<false>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_done[raw] = true;
+  }
+  const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+  const int pairs_fit = max_pairs(raw_int32, num_sms);
+  const int pairs = tiles < pairs_fit ? tiles : pairs_fit;
+  if (raw_int32)
+    k_gemm_i8_tcgen05<true><<<2 * pairs, THREADS, SMEM_ALLOC, st>>>(maps, a);
+  else
+    k_gemm_i8_tcgen05<false><<<2 * pairs, THREADS, SMEM_ALLOC, st>>>(maps, a);
   return cudaGetLastError();
 }
 

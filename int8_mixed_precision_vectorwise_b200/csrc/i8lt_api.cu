@@ -71,18 +71,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major [rows, inner] matrix, boxes of box_inner x box_rows elements, 128B swizzle.
+// Row-major [rows, inner] matrix, boxes of box_inner x box_rows elements.
 bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
-               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {row_stride_bytes};
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int num_sms() {
@@ -112,24 +112,31 @@ i8_status check_gemm_operands(const void* A, const void* B, int M, int N, int K)
   return I8_OK;
 }
 
-i8_status run_gemm(const int8_t* A, const int8_t* B, int M, int N, int K, const GemmArgs& args, bool raw,
+i8_status run_gemm(const int8_t* A, const int8_t* B, int M, int N, int K, GemmArgs args, bool raw,
                    const __half* XO, const __half* WO, int ld_o, cudaStream_t st) {
-  CUtensorMap tmA, tmB, tmXO, tmWO;
-  std::memset(&tmXO, 0, sizeof(tmXO));
-  std::memset(&tmWO, 0, sizeof(tmWO));
-  if (!encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, i8lt::kGemmBKBytes, i8lt::kGemmBM) ||
-      !encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, i8lt::kGemmBKBytes, i8lt::kGemmBN))
+  i8lt::GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const uint32_t kbk = i8lt::kGemmBKBytes;
+  if (!encode_2d(&maps.A, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, kbk, i8lt::kGemmBM) ||
+      !encode_2d(&maps.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, kbk, i8lt::kGemmBN / 2))
     return I8_ERR_CUDA;
   if (XO != nullptr && WO != nullptr && ld_o > 0) {
-    if (!encode_2d(&tmXO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, XO, ld_o, M, static_cast<uint64_t>(ld_o) * 2, 64,
-                   i8lt::kGemmBM) ||
-        !encode_2d(&tmWO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, WO, ld_o, N, static_cast<uint64_t>(ld_o) * 2, 64,
-                   i8lt::kGemmBN))
+    const uint64_t ld_bytes = static_cast<uint64_t>(ld_o) * 2;
+    if (!encode_2d(&maps.XO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, XO, ld_o, M, ld_bytes, 64, i8lt::kGemmBM) ||
+        !encode_2d(&maps.WO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, WO, ld_o, N, ld_bytes, 64, i8lt::kGemmBN / 2))
       return I8_ERR_CUDA;
+  }
+  args.tma_store = 0;
+  if (!raw && N % 8 == 0) {
+    // fp16 rows must be 16-byte multiples for the TMA store; otherwise plain stores
+    if (!encode_2d(&maps.Out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, args.out, N, M, static_cast<uint64_t>(N) * 2,
+                   i8lt::kGemmOutBox, i8lt::kGemmOutBox, CU_TENSOR_MAP_SWIZZLE_64B))
+      return I8_ERR_CUDA;
+    args.tma_store = 1;
   }
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
-  return cuda_status(i8lt::launch_gemm(tmA, tmB, tmXO, tmWO, args, raw, sms, st));
+  return cuda_status(i8lt::launch_gemm(maps, args, raw, sms, st));
 }
 
 }  // namespace
@@ -202,6 +209,9 @@ i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_ha
   a.out = reinterpret_cast<__half*>(out);
   a.n_used = with_o ? reinterpret_cast<const int32_t*>(w.hdr + 1) : nullptr;
   a.out_cap = cap;
+  a.XO = with_o ? w.XO : nullptr;
+  a.WO = with_o ? w.WO : nullptr;
+  a.ld_o = L.ld_o;
   a.status = w.hdr;
   a.wait_limit_ns = kWaitLimitNs;
   return run_gemm(w.CA, CB, M, N, K, a, false, with_o ? w.XO : nullptr, with_o ? w.WO : nullptr, L.ld_o, st);

@@ -34,17 +34,33 @@ struct GemmArgs {
   int out_cap;             // capacity of the gathered outlier operands (columns)
   uint32_t* status;        // device status word, or nullptr
   uint64_t wait_limit_ns;  // bound on every pipeline wait
+  int tma_store;           // fused mode: write out through tmOut (needs N % 8 == 0)
+  // Few outlier columns (n_used <= kSmallOutliers) are added by the epilogue
+  // with warp-level MMAs straight from the gathered operands:
+  const __half* XO;        // [M, ld_o] gathered X[:, O] (zero padded)
+  const __half* WO;        // [N, ld_o] fp16(CB[:, O]) (zero padded)
+  int ld_o;
 };
 
-// tmA: CA [M, K] int8; tmB: CB [N, K] int8; tmXO / tmWO: gathered fp16 outlier
-// operands [M, ld] / [N, ld] (unused unless n_used != nullptr).
-cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmXO,
-                        const CUtensorMap& tmWO, const GemmArgs& a, bool raw_int32, int num_sms, cudaStream_t st);
+// Tensor maps of one GEMM call.  A: CA [M, K] int8 (box 128 rows x 128 B).
+// B: CB [N, K] int8 (box 128 rows x 128 B).  XO / WO: gathered fp16 outlier
+// operands [M, ld] / [N, ld] (boxes 128 x 64 fp16; used for more than
+// kSmallOutliers columns).  Out: out [M, N] fp16 (box 32 x 32; unused unless
+// tma_store).
+struct GemmMaps {
+  CUtensorMap A, B, XO, WO, Out;
+};
+
+constexpr int kSmallOutliers = 16;
+
+// The kernel runs on CTA pairs.
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, bool raw_int32, int num_sms, cudaStream_t st);
 
 // Box sizes the tensor maps above must be encoded with.
-constexpr int kGemmBM = 128;       // rows of A per tile
-constexpr int kGemmBN = 256;       // rows of B per tile
-constexpr int kGemmBKBytes = 128;  // bytes of K per pipeline stage
+constexpr int kGemmBM = 128;        // rows of A per CTA (a CTA pair covers 256 rows)
+constexpr int kGemmBN = 256;        // output columns per pair tile (each CTA loads 128 rows of B)
+constexpr int kGemmBKBytes = 128;   // bytes of K per pipeline stage
+constexpr int kGemmOutBox = 32;     // output box: 32 columns x 32 rows (64-byte swizzle)
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 

@@ -4,7 +4,7 @@
 //                       "Improved kernels for inference", int8_vectorwise_quant)
 //   k_zero_outlier_cols zero the outlier columns of the codes (the fp16 path owns them)
 //   k_outlier_prepare   bitmap -> sorted outlier column list (state.idx), zero CA
-//                       columns, gather X[:, O] and fp16(CB[:, O]) for the fp16 MMA
+//                       columns, gather X[:, O] and fp16(CB[:, O]) for the outlier product
 //   k_mm_dequant        int32 -> fp16 with row x column scales / 127^2 + bias
 //   k_dequant           int8 weight -> fp16 ("Next steps": int8 dequantize op)
 #include <cuda_fp16.h>
