@@ -161,6 +161,68 @@ __global__ void __launch_bounds__(256) k_quant_rows_stream(const __half* __restr
   for (int vi = threadIdx.x; vi < nvec; vi += 256) cr[vi] = quant8(xr[vi], r);
 }
 
+// Persistent warp-per-row variant for many rows.  Pass 1 streams the row from
+// HBM, U 16-byte loads per lane in flight, and reduces |x| with packed fp16
+// max (exact: the max of fp16 values is one of them); only vectors whose max
+// reaches the threshold take the per-element fp32 path that separates
+// outliers.  Pass 2 re-reads the row (now in L2) and writes the codes.  No
+// block-level synchronisation: every warp walks its own rows.
+template <int U>
+__global__ void __launch_bounds__(256) k_quant_rows_warp(const __half* __restrict__ X, int M, int K, float tau,
+                                                         int8_t* __restrict__ CA, float* __restrict__ SCA,
+                                                         uint32_t* __restrict__ bitmap) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  const int nvec = K >> 3;
+  const bool use_tau = tau > 0.f;
+  for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < M; row += nwarps) {
+    const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * K);
+    float amax = 0.f;
+    for (int base = 0; base < nvec; base += 32 * U) {  // uniform trip count for the warp votes
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int vi = base + u * 32 + lane;
+        v[u] = vi < nvec ? __ldg(xr + vi) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const __half2* h = reinterpret_cast<const __half2*>(&v[u]);
+        const __half2 m = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
+        const float vmax = fmaxf(__low2float(m), __high2float(m));
+        const bool hot = use_tau && vmax >= tau;  // some element of this vector is an outlier
+        if (__any_sync(kFull, hot)) {
+          uint32_t big = 0;
+          float keep = 0.f;
+          if (hot) scan8(v[u], tau, true, keep, big); else keep = vmax;
+          amax = fmaxf(amax, keep);
+          publish_outliers(big, base + u * 32 + lane, bitmap);
+        } else {
+          amax = fmaxf(amax, vmax);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+    const float r = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    if (lane == 0) SCA[row] = amax;
+    uint2* cr = reinterpret_cast<uint2*>(CA + static_cast<size_t>(row) * K);
+    for (int base = 0; base < nvec; base += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int vi = base + u * 32 + lane;
+        if (vi < nvec) v[u] = __ldcs(xr + vi);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int vi = base + u * 32 + lane;
+        if (vi < nvec) cr[vi] = quant8(v[u], r);
+      }
+    }
+  }
+}
+
 // Zero every outlier column of CA straight from the bitmap (one warp per row).
 __global__ void __launch_bounds__(256) k_zero_outlier_cols(const uint32_t* __restrict__ bitmap, int M, int K,
                                                            int8_t* __restrict__ CA) {
@@ -333,7 +395,21 @@ __global__ void __launch_bounds__(256) k_dequant(const int8_t* __restrict__ CB, 
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
-                              cudaStream_t st) {
+                              uint32_t* status, int num_sms, cudaStream_t st) {
+  (void)status;
+  // Many rows: persistent warps, one row each at a time.
+  if (M >= 8 * num_sms) {
+    static int blocks_per_sm = 0;
+    if (blocks_per_sm == 0) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, k_quant_rows_warp<8>, 256, 0) !=
+              cudaSuccess ||
+          blocks_per_sm <= 0)
+        blocks_per_sm = 4;
+    }
+    const int warps = (M + 0) < num_sms * blocks_per_sm * 8 ? M : num_sms * blocks_per_sm * 8;
+    k_quant_rows_warp<8><<<(warps + 7) / 8, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
+    return cudaGetLastError();
+  }
   const int nvec = K / 8;
   if (nvec <= 32 * 8) {
     k_quant_rows<32, 8><<<(M + 7) / 8, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
