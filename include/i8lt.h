@@ -169,6 +169,10 @@ I8_API i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const
  *     operands X[:, O] and CB[:, O].
  *   i8_linear8bit_matmul_dequant: the tensor-core GEMM with the fused
  *     dequant / bias / outlier epilogue, reading the prepared workspace.
+ *     Enqueue it right after i8_linear8bit_prepare on the same stream (events
+ *     may sit in between, other kernels may not): it is launched as a
+ *     programmatic dependent of the preparation and, for few tokens, starts
+ *     streaming CB before the preparation has finished.
  */
 I8_API i8_status i8_linear8bit_prepare(const i8_half* X, const int8_t* CB, int M, int N, int K,
                                        float threshold, void* workspace, size_t workspace_bytes,

@@ -102,15 +102,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int num_n = (N + BN - 1) / BN;
   const int tiles = num_m * num_n;
   const int kb_int = (K + BK - 1) / BK;
-  int n_used = 0;
-  if (!RAW && p.n_used != nullptr) n_used = min(max(*p.n_used, 0), p.out_cap);
-  // Few outlier columns are added by the epilogue on CUDA cores (a rank-n
-  // update) so the TMEM accumulators stay double-buffered; more go through an
-  // fp16 MMA into a second accumulator.
-  const bool small_o = n_used > 0 && n_used <= SMALL_O && p.XO != nullptr && p.WO != nullptr;
-  const int kb_out = small_o ? 0 : (n_used + 63) / 64;
-  const int kb_all = kb_int + kb_out;
-  const bool dbl = kb_out == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -128,10 +119,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm.A);
     tma_prefetch_desc(&tm.B);
-    if (kb_out > 0) {
-      tma_prefetch_desc(&tm.XO);
-      tma_prefetch_desc(&tm.WO);
-    }
     if (!RAW && p.tma_store) tma_prefetch_desc(&tm.Out);
   }
   if (warp == 1) {
@@ -142,6 +129,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();  // barriers initialised and TMEM allocated in both CTAs of the pair
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
+
+  // The kernel may be launched while the kernel before it (the outlier
+  // preparation) still runs: everything below reads what that kernel and the
+  // quantiser wrote, so wait for them here (a no-op without that overlap).
+  pdl_wait();
+  int n_used = 0;
+  if (!RAW && p.n_used != nullptr) n_used = min(max(*p.n_used, 0), p.out_cap);
+  // Up to 16 outlier columns are added by the epilogue with warp MMAs so the
+  // TMEM accumulators stay double-buffered; more go through tcgen05 fp16 MMAs
+  // into a second accumulator.
+  const bool small_o = n_used > 0 && n_used <= SMALL_O && p.XO != nullptr && p.WO != nullptr;
+  const int kb_out = small_o ? 0 : (n_used + 63) / 64;
+  const int kb_all = kb_int + kb_out;
+  const bool dbl = kb_out == 0;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -489,11 +490,18 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, bool raw_int32,
   const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
   const int pairs_fit = max_pairs(raw_int32, num_sms);
   const int pairs = tiles < pairs_fit ? tiles : pairs_fit;
-  if (raw_int32)
-    k_gemm_i8_tcgen05<true><<<2 * pairs, THREADS, SMEM_ALLOC, st>>>(maps, a);
-  else
-    k_gemm_i8_tcgen05<false><<<2 * pairs, THREADS, SMEM_ALLOC, st>>>(maps, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return raw_int32 ? cudaLaunchKernelEx(&cfg, k_gemm_i8_tcgen05<true>, maps, a)
+                   : cudaLaunchKernelEx(&cfg, k_gemm_i8_tcgen05<false>, maps, a);
 }
 
 // ------------------------------------------------------------------ self test

@@ -26,17 +26,23 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t hdr, bitmap, idx, sca, ca, xo, wo, total;
-  int ld_o;  // row stride (fp16 elements) of the gathered outlier operands
+  size_t hdr, bitmap, counters, idx, sca, ca, xo, wo, partials, total;
+  size_t clear_bytes;  // prefix cleared by every call: header, bitmap, split-K counters
+  int ld_o;            // row stride (fp16 elements) of the gathered outlier operands
+  bool decode;         // few tokens: the decode GEMM (split-K partials, no W_O gather)
 };
 
 bool ws_layout(int M, int N, int K, int cap, WsLayout* L) {
   if (M <= 0 || N <= 0 || K <= 0 || cap < 0) return false;
+  L->decode = M <= i8lt::kDecodeMaxTokens;
   size_t off = 0;
   L->hdr = off;
   off += kHdrBytes;
   L->bitmap = off;
   off += align256(static_cast<size_t>((K + 31) / 32) * 4);
+  L->counters = off;
+  off += L->decode ? align256(static_cast<size_t>((N + 127) / 128) * 4 * 4) : 0;
+  L->clear_bytes = off;
   L->idx = off;
   off += align256(static_cast<size_t>(cap > 0 ? cap : 1) * 4);
   L->sca = off;
@@ -47,7 +53,9 @@ bool ws_layout(int M, int N, int K, int cap, WsLayout* L) {
   L->xo = off;
   off += align256(static_cast<size_t>(M) * L->ld_o * 2);
   L->wo = off;
-  off += align256(static_cast<size_t>(N) * L->ld_o * 2);
+  off += L->decode ? 0 : align256(static_cast<size_t>(N) * L->ld_o * 2);
+  L->partials = off;
+  off += L->decode ? align256(static_cast<size_t>(i8lt::decode_slots(N, K)) * i8lt::kDecodeMaxTokens * N * 4) : 0;
   L->total = off;
   return true;
 }
@@ -161,6 +169,8 @@ i8_status check_forward(const i8_half* X, const int8_t* CB, const float* SCB, co
 struct WsPtrs {
   uint32_t* hdr;
   uint32_t* bitmap;
+  int32_t* counters;
+  int32_t* partials;
   int32_t* idx;
   float* SCA;
   int8_t* CA;
@@ -171,6 +181,7 @@ struct WsPtrs {
 WsPtrs ws_ptrs(void* workspace, const WsLayout& L) {
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return WsPtrs{reinterpret_cast<uint32_t*>(ws + L.hdr), reinterpret_cast<uint32_t*>(ws + L.bitmap),
+                reinterpret_cast<int32_t*>(ws + L.counters), reinterpret_cast<int32_t*>(ws + L.partials),
                 reinterpret_cast<int32_t*>(ws + L.idx),  reinterpret_cast<float*>(ws + L.sca),
                 reinterpret_cast<int8_t*>(ws + L.ca),    reinterpret_cast<__half*>(ws + L.xo),
                 reinterpret_cast<__half*>(ws + L.wo)};
@@ -183,16 +194,15 @@ i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int 
   const bool outliers = threshold > 0.f;
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
-  // status word, counts and the bitmap are contiguous: one memset clears them
-  if (cudaMemsetAsync(workspace, 0, L.bitmap + static_cast<size_t>((K + 31) / 32) * 4, st) != cudaSuccess)
-    return I8_ERR_CUDA;
+  // status word, counts, bitmap and split-K counters are contiguous: one memset clears them
+  if (cudaMemsetAsync(workspace, 0, L.clear_bytes, st) != cudaSuccess) return I8_ERR_CUDA;
   i8_status s = cuda_status(
       i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr, w.hdr, sms, st));
   if (s != I8_OK || !outliers) return s;
   return cuda_status(i8lt::launch_outlier_prepare(w.bitmap, K, cap, reinterpret_cast<int32_t*>(w.hdr + 2),
                                                   reinterpret_cast<int32_t*>(w.hdr + 1), w.idx, w.hdr, w.CA, Xh, M,
-                                                  cap > 0 ? w.XO : nullptr, CB, N, cap > 0 ? w.WO : nullptr, L.ld_o,
-                                                  sms, st));
+                                                  cap > 0 ? w.XO : nullptr, CB, N,
+                                                  (cap > 0 && !L.decode) ? w.WO : nullptr, L.ld_o, sms, st));
 }
 
 i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N, int K,
@@ -200,6 +210,37 @@ i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_ha
                                  cudaStream_t st) {
   const WsPtrs w = ws_ptrs(workspace, L);
   const bool with_o = threshold > 0.f && cap > 0;
+  if (L.decode) {
+    i8lt::DecodeArgs d{};
+    d.M = M;
+    d.N = N;
+    d.K = K;
+    d.SCA = w.SCA;
+    d.SCB = SCB;
+    d.bias = reinterpret_cast<const __half*>(bias);
+    d.out = reinterpret_cast<__half*>(out);
+    d.CB = CB;
+    d.idx = w.idx;
+    d.n_used = with_o ? reinterpret_cast<const int32_t*>(w.hdr + 1) : nullptr;
+    d.out_cap = cap;
+    d.XO = w.XO;
+    d.ld_o = L.ld_o;
+    d.partials = w.partials;
+    d.counters = w.counters;
+    d.status = w.hdr;
+    d.wait_limit_ns = kWaitLimitNs;
+    CUtensorMap tmW, tmC;
+    if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, CB, K, N, K, 128, 128) ||
+        !encode_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.CA, K, M, K, 128, i8lt::kDecodeMaxTokens))
+      return I8_ERR_CUDA;
+    const int sms = num_sms();
+    if (sms <= 0) return I8_ERR_CUDA;
+    const int boxes = 4;  // 512 bytes of each weight row per pipeline stage
+    const int total = ((N + 127) / 128) * ((K + 128 * boxes - 1) / (128 * boxes));
+    int grid = sms < i8lt::kDecodeMaxGrid ? sms : i8lt::kDecodeMaxGrid;
+    if (grid > total) grid = total;
+    return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, grid, boxes, st));
+  }
   GemmArgs a{};
   a.M = M;
   a.N = N;

@@ -63,6 +63,40 @@ constexpr int kGemmBN = 256;        // output columns per pair tile (each CTA lo
 constexpr int kGemmBKBytes = 128;   // bytes of K per pipeline stage
 constexpr int kGemmOutBox = 32;     // output box: 32 columns x 32 rows (64-byte swizzle)
 
+// Few-token (decode) GEMM: weights are the wide MMA operand, tokens padded to 16.
+constexpr int kDecodeMaxTokens = 16;
+
+struct DecodeArgs {
+  int M, N, K;               // M = tokens (<= kDecodeMaxTokens)
+  const float* SCA;          // [M]
+  const float* SCB;          // [N]
+  const __half* bias;        // [N] or nullptr
+  __half* out;               // [M, N]
+  const int8_t* CB;          // [N, K] (outlier columns are read from it directly)
+  const int32_t* idx;        // sorted outlier columns
+  const int32_t* n_used;     // device count of outlier columns, or nullptr
+  int out_cap;
+  const __half* XO;          // [M, ld_o] gathered X[:, O]
+  int ld_o;
+  int32_t* partials;         // [slots][16][N] split-K partial sums
+  int32_t* counters;         // [ceil(N/128) * 4], zero on entry
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+
+// Partial-sum slots the decode GEMM needs for these sizes (grid <= kDecodeMaxGrid).
+constexpr int kDecodeMaxGrid = 256;
+inline int decode_slots(int N, int K) {
+  const int kb = (K + 127) / 128, ntiles = (N + 127) / 128;
+  const int s = kDecodeMaxGrid / ntiles + 2;
+  return s < kb ? s : kb;
+}
+
+// tmW: CB [N, K] int8, box 128 rows x 128 B; tmC: CA [M, K] int8, box 16 rows x 128 B.
+// boxes_per_stage: 128-byte K boxes per pipeline stage (1, 2 or 4).
+cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
+                               int boxes_per_stage, cudaStream_t st);
+
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 
 }  // namespace i8lt

@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(256) k_quant_rows(const __half* __restrict__ X
                                                     int8_t* __restrict__ CA, float* __restrict__ SCA,
                                                     uint32_t* __restrict__ bitmap) {
   static_assert(G % 32 == 0 && 256 % G == 0, "group size");
+  pdl_launch_dependents();
   constexpr int ROWS = 256 / G;
   constexpr int WPR = G / 32;  // warps per row
   __shared__ float red[8];
@@ -136,6 +137,7 @@ __global__ void __launch_bounds__(256) k_quant_rows_stream(const __half* __restr
                                                            float tau, int8_t* __restrict__ CA,
                                                            float* __restrict__ SCA, uint32_t* __restrict__ bitmap) {
   __shared__ float red[8];
+  pdl_launch_dependents();
   const int row = blockIdx.x;
   const int nvec = K >> 3;
   const bool use_tau = tau > 0.f;
@@ -171,6 +173,7 @@ template <int U>
 __global__ void __launch_bounds__(256) k_quant_rows_warp(const __half* __restrict__ X, int M, int K, float tau,
                                                          int8_t* __restrict__ CA, float* __restrict__ SCA,
                                                          uint32_t* __restrict__ bitmap) {
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * (blockDim.x >> 5);
   const int nvec = K >> 3;
@@ -260,6 +263,8 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
   extern __shared__ int32_t idx_s[];
   __shared__ int32_t warp_base[8];
   __shared__ int32_t s_total;
+  pdl_launch_dependents();
+  pdl_wait();  // the bitmap and codes come from the quantiser
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwords = (K + 31) >> 5;
   const int per = (nwords + 255) / 256;
@@ -441,9 +446,18 @@ cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32
   const int rows = ((XO || CA) ? M : 0) + (WO ? N : 0);
   const int blocks = max(1, min((rows + 7) / 8, num_sms * 4));
   const size_t smem = static_cast<size_t>(max(cap, 1)) * sizeof(int32_t);
-  k_outlier_prepare<<<blocks, 256, smem, st>>>(bitmap, K, cap, total_out, used_out, idx_out, status, CA, X, M, XO,
-                                               CB, N, WO, ld_o);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_outlier_prepare, bitmap, K, cap, total_out, used_out, idx_out, status, CA, X, M,
+                            XO, CB, N, WO, ld_o);
 }
 
 cudaError_t launch_mm_dequant(const int32_t* C, const float* SCA, const float* SCB, const __half* bias, int M,
