@@ -11,17 +11,22 @@
 // few words", with the int8_linear_matmul / int8_mm_dequant ops of
 // "LLM.int8() Refactoring: Part 1", section "Deprecations").
 //
-// Work split ("stream-K"): the (128-row tile, 128-byte k-block) grid is cut
-// into one contiguous range of k-blocks per CTA, so every SM streams the same
-// number of weight bytes.  A tile split across CTAs leaves int32 partials in a
-// workspace slot per contributing CTA; per 32-row quarter, a counter tells
-// the last contributor, which sums the partials and writes the outputs.
-// Outlier columns (CA already zeroed there) are added by that last warp on
-// CUDA cores from the gathered X[:, O] and the int8 weight columns.
+// Work split ("stream-K"): the (128-row tile, k-stage) grid is cut into one
+// contiguous range of stages per CTA, so every SM streams the same number of
+// weight bytes.  A tile split across CTAs leaves int32 partials (and fp32
+// partials of the outlier term) in a workspace slot per contributing CTA; per
+// 32-row quarter, a counter tells the last contributor, which sums them and
+// writes the outputs.
 //
-// Block = 6 warps: TMA producer, MMA issuer (+ TMEM owner), 4 epilogue warps
-// (one per 32-lane TMEM quadrant).  A 12-stage ring keeps ~200 KB of weights
-// in flight per SM.
+// The outlier columns (CA already zeroed there) are added from the weight
+// tiles while they sit in shared memory: every column is streamed exactly
+// once, by the CTA whose k-range holds it, so the fp16 term costs no extra
+// HBM traffic.
+//
+// Block = 7 warps: TMA producer, MMA issuer (+ TMEM owner), 4 epilogue warps
+// (one per 32-lane TMEM quadrant), and the outlier warp.  A stage is released
+// when both the MMAs and the outlier warp are done with it.  A 3-stage ring of
+// 72 KB stages keeps ~216 KB of weights in flight per SM.
 #include <cuda_fp16.h>
 
 #include "kernels.cuh"
@@ -34,20 +39,23 @@ namespace {
 constexpr int DM = 128;                    // weight rows per tile (MMA M)
 constexpr int DT = kDecodeMaxTokens;       // token columns (MMA N), zero padded
 constexpr int DK = 128;                    // bytes of K per swizzle atom / TMA box
-constexpr int DTHREADS = 64 + 128;
+constexpr int DTHREADS = 64 + 128 + 32;
 constexpr int DA_BYTES = DM * DK;          // 16 KB of weights per box
 constexpr int DB_BYTES = DT * DK;          // 2 KB of codes per box
 constexpr int DBOX_BYTES = DA_BYTES + DB_BYTES;
 constexpr uint32_t DTMEM_COLS = 32;        // two 16-column accumulators
 
 // C boxes (C x 128 bytes of K) per pipeline stage, DRING bytes of ring.
+constexpr int DS_BYTES = DT * DM * 4;      // one segment's outlier term, fp32 [token][row]
+
 template <int C>
 struct DecodeCfg {
   static constexpr int STAGE_BYTES = C * DBOX_BYTES;
   static constexpr int STAGES = (12 * DBOX_BYTES) / STAGE_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 5;
+  static constexpr int NUM_BARS = 2 * STAGES + 7;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int MISC_OFF = BAR_OFF + ((NUM_BARS * 8 + 15) / 16) * 16;
+  static constexpr int DS_OFF = BAR_OFF + ((NUM_BARS * 8 + 15) / 16) * 16;
+  static constexpr int MISC_OFF = DS_OFF + DS_BYTES;
   static constexpr int SMEM_ALLOC = MISC_OFF + 16 + 1024;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
@@ -89,6 +97,9 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   uint64_t* acc_full = empty + DSTAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
   uint64_t* mma_done = acc_empty + 2;
+  uint64_t* d_full = mma_done + 1;       // the outlier term of a segment is in d_s
+  uint64_t* d_empty = d_full + 1;        // ... and has been read by the 4 epilogue warps
+  float* d_s = reinterpret_cast<float*>(smem + Cfg::DS_OFF);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Cfg::MISC_OFF);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -105,13 +116,15 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < DSTAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 2);  // the MMAs' commit and the outlier warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);
     }
     mbar_init(mma_done, 1);
+    mbar_init(d_full, 1);
+    mbar_init(d_empty, 4);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -223,18 +236,96 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       drain_wait_d(mma_done, 0, p.wait_limit_ns);
     }
     __syncwarp();
+  } else if (warp == 6) {
+    // ---------------------------------------------------------------- outlier warp
+    // Lane l owns rows l, l+32, l+64, l+96 of the tile.  Every stage is waited
+    // for and released; stages holding outlier columns add X[t, j] * CB[n, j]
+    // (weights read from the swizzled tile) into a per-segment fp32 sum that
+    // is handed to the epilogue through d_s at the segment's end.
+    pdl_wait();  // outlier list and gathered X come from the preceding kernel
+    const int n_used = p.n_used != nullptr ? min(max(*p.n_used, 0), p.out_cap) : 0;
+    int stage = 0;
+    uint32_t phase = 0;
+    int segi = 0;
+    bool ok = true;
+    SegIter seg(kb, start, end);
+    int tile, k0, k1;
+    while (ok && seg.next(tile, k0, k1)) {
+      float d[4][DT];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int t = 0; t < DT; ++t) d[i][t] = 0.f;
+      // first outlier column at or after this segment's k-range
+      int cur = 0;
+      while (cur < n_used && __ldg(p.idx + cur) < k0 * DKS) ++cur;
+      for (int k = k0; k < k1; ++k) {
+        int got = 0;
+        if (lane == 0) got = mbar_wait_bounded(&full[stage], phase, s_abort, p.status, p.wait_limit_ns) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* sa = smem + stage * DSTAGE_BYTES;
+        while (cur < n_used) {
+          const int j = __ldg(p.idx + cur);
+          if (j >= (k + 1) * DKS) break;
+          const int kk = j - k * DKS;                // byte within the stage
+          const int box = kk >> 7, b = kk & 127;     // 128-byte box, byte within the row
+          float x[DT];
+#pragma unroll
+          for (int t = 0; t < DT; ++t) x[t] = t < T ? __half2float(p.XO[static_cast<size_t>(t) * p.ld_o + cur]) : 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = lane + 32 * i;             // 128B swizzle: 16-byte chunk q of row r sits at q ^ (r % 8)
+            const float w = static_cast<float>(static_cast<int8_t>(
+                sa[box * DA_BYTES + r * 128 + ((((b >> 4) ^ (r & 7))) << 4) + (b & 15)]));
+#pragma unroll
+            for (int t = 0; t < DT; ++t) d[i][t] = fmaf(x[t], w, d[i][t]);
+          }
+          ++cur;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == DSTAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      // hand the segment's sum to the epilogue (once it has read the previous one)
+      if (segi > 0) {
+        int got = 0;
+        if (lane == 0) got = mbar_wait_bounded(d_empty, static_cast<uint32_t>(segi - 1) & 1u, s_abort, p.status,
+                                               p.wait_limit_ns) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      }
+      if (n_used > 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int t = 0; t < DT; ++t) d_s[t * DM + lane + 32 * i] = d[i][t];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(d_full);
+      ++segi;
+    }
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quad = warp & 3;  // TMEM lanes = weight rows quad*32 .. +31 of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    pdl_wait();  // scales, outlier list and gathered inputs come from the preceding kernels
+    pdl_wait();  // scales and the outlier count come from the preceding kernel
     const int n_used = p.n_used != nullptr ? min(max(*p.n_used, 0), p.out_cap) : 0;
+    const size_t dpart = static_cast<size_t>(p.slots) * DT * N;  // fp32 partials follow the int32 ones
     int it = 0;
     SegIter seg(kb, start, end);
     int tile, k0, k1;
     while (seg.next(tile, k0, k1)) {
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int n = tile * DM + quad * 32 + lane;
+      const float sb = n < N ? __ldg(p.SCB + n) : 0.f;
+      const float bv = (n < N && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
       int ok = 0;
       if (lane == 0) ok = mbar_wait_bounded(&acc_full[buf], use & 1u, s_abort, p.status, p.wait_limit_ns) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -245,10 +336,18 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);  // the accumulator is in registers now
+      // this segment's outlier term (the outlier warp is done with the segment by now or soon)
+      ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded(d_full, static_cast<uint32_t>(it) & 1u, s_abort, p.status, p.wait_limit_ns) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      float d[DT];
+#pragma unroll
+      for (int t = 0; t < DT; ++t) d[t] = (n_used > 0 && t < T) ? d_s[t * DM + quad * 32 + lane] : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(d_empty);
       ++it;
 
-      const int n = tile * DM + quad * 32 + lane;
-      // contributors of this tile: CTAs whose k-block range meets it
+      // contributors of this tile: CTAs whose k-stage range meets it
       const int first = (tile * kb) / per;
       const int last_cta = ((tile + 1) * kb - 1) / per;
       const int nseg = last_cta - first + 1;
@@ -256,10 +355,14 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       if (nseg > 1) {
         const int slot = static_cast<int>(blockIdx.x) - first;
         int32_t* part = p.partials + (static_cast<size_t>(slot) * DT) * N;
+        float* dp = reinterpret_cast<float*>(p.partials + dpart) + (static_cast<size_t>(slot) * DT) * N;
         if (n < N) {
 #pragma unroll
-          for (int t = 0; t < DT; ++t)
-            if (t < T) __stcg(part + static_cast<size_t>(t) * N + n, static_cast<int32_t>(c[t]));
+          for (int t = 0; t < DT; ++t) {
+            if (t >= T) break;
+            __stcg(part + static_cast<size_t>(t) * N + n, static_cast<int32_t>(c[t]));
+            if (n_used > 0) __stcg(dp + static_cast<size_t>(t) * N + n, d[t]);
+          }
         }
         __threadfence();
         __syncwarp();
@@ -269,39 +372,34 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         if (finalize) {
           __threadfence();
           if (n < N) {
+            // the other contributors' slots: all tokens of a slot in flight at once
+            int32_t acc[DT];
 #pragma unroll
-            for (int t = 0; t < DT; ++t) {
-              if (t >= T) break;
-              int32_t sum = 0;
-              for (int sl = 0; sl < nseg; ++sl)
-                sum += __ldcg(p.partials + (static_cast<size_t>(sl) * DT + t) * N + n);
-              c[t] = static_cast<uint32_t>(sum);
+            for (int t = 0; t < DT; ++t) acc[t] = static_cast<int32_t>(c[t]);
+            for (int sl = 0; sl < nseg; ++sl) {
+              if (sl == slot) continue;
+              const int32_t* src = p.partials + (static_cast<size_t>(sl) * DT) * N + n;
+              const float* dsrc = reinterpret_cast<const float*>(p.partials + dpart) + (static_cast<size_t>(sl) * DT) * N + n;
+              int32_t v[DT];
+              float dv[DT];
+#pragma unroll
+              for (int t = 0; t < DT; ++t) {
+                v[t] = t < T ? __ldcg(src + static_cast<size_t>(t) * N) : 0;
+                dv[t] = (n_used > 0 && t < T) ? __ldcg(dsrc + static_cast<size_t>(t) * N) : 0.f;
+              }
+#pragma unroll
+              for (int t = 0; t < DT; ++t) {
+                acc[t] += v[t];
+                d[t] += dv[t];
+              }
             }
+#pragma unroll
+            for (int t = 0; t < DT; ++t) c[t] = static_cast<uint32_t>(acc[t]);
           }
         }
       }
       if (!finalize || n >= N) continue;
-      // dequant + bias + outlier columns for (t, n), t < T
-      const float sb = __ldg(p.SCB + n);
-      const float bv = p.bias != nullptr ? __half2float(p.bias[n]) : 0.f;
-      float d[DT];
-#pragma unroll
-      for (int t = 0; t < DT; ++t) d[t] = 0.f;
-      const int8_t* cbrow = p.CB + static_cast<size_t>(n) * K;
-      for (int j0 = 0; j0 < n_used; j0 += 16) {
-        // issue up to 16 outlier-weight loads at once, then use them
-        float w[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj)
-          w[jj] = j0 + jj < n_used ? static_cast<float>(cbrow[__ldg(p.idx + j0 + jj)]) : 0.f;
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          if (j0 + jj >= n_used) break;
-#pragma unroll
-          for (int t = 0; t < DT; ++t)
-            if (t < T) d[t] = fmaf(__half2float(p.XO[static_cast<size_t>(t) * p.ld_o + j0 + jj]), w[jj], d[t]);
-        }
-      }
+      // dequant + bias + outlier term for (t, n), t < T
 #pragma unroll
       for (int t = 0; t < DT; ++t) {
         if (t >= T) break;

@@ -17,6 +17,10 @@
 // the leader CTA issues one M=256 MMA over both halves.  Each CTA's TMEM holds
 // the accumulator rows of its half.
 //
+// Tiles are handed to pairs round-robin; when the last round would leave
+// more than half of the pairs idle, its tiles are split into 256 x 128 halves
+// (MMA N = 128), so that round takes about half the time of a full one.
+//
 // Block = 10 warps: warp 0 issues TMA loads (one lane), warp 1 owns TMEM and,
 // in the leader, issues tcgen05.mma (one lane); warps 2-9 run the epilogue
 // (two warps per 32-lane TMEM quadrant, one per 128-column half).  K streams
@@ -71,6 +75,30 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   mbar_wait_bounded(bar, parity, &never, nullptr, limit_ns);
 }
 
+// Work units of a pair: tiles [0, full_units) are whole 256 x 256 tiles; past
+// them each remaining tile is cut into two 256 x 128 halves, so a last wave
+// that would keep at most half of the pairs busy takes half as long (and a
+// grid with fewer tiles than half the pairs runs twice as many CTAs).
+struct Units {
+  int full_units, units;
+  __device__ Units(int tiles, int npairs) {
+    const int waves = tiles / npairs, rem = tiles - waves * npairs;
+    const bool split = rem > 0 && 2 * rem <= npairs;
+    full_units = split ? waves * npairs : tiles;
+    units = split ? full_units + 2 * rem : tiles;
+  }
+  // tile of unit u and which column half of it (-1: the whole tile)
+  __device__ void at(int u, int& tile, int& half) const {
+    if (u < full_units) {
+      tile = u;
+      half = -1;
+    } else {
+      tile = full_units + ((u - full_units) >> 1);
+      half = (u - full_units) & 1;
+    }
+  }
+};
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -102,6 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int num_n = (N + BN - 1) / BN;
   const int tiles = num_m * num_n;
   const int kb_int = (K + BK - 1) / BK;
+  const Units U(tiles, npairs);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -151,9 +180,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t filled = 0, fill_parity = 0;  // leader: per stage, ever filled / parity of the last fill
-      for (int tile = pair; tile < tiles && !*s_abort; tile += npairs) {
+      for (int u = pair; u < U.units && !*s_abort; u += npairs) {
+        int tile, half;
+        U.at(u, tile, half);
         const int m0 = (tile % num_m) * (2 * BM) + static_cast<int>(rank) * BM;
-        const int nb0 = (tile / num_m) * BN + static_cast<int>(rank) * BNH;
+        // a half tile's 128 columns come as 64 B rows per CTA (the box still
+        // carries 128 rows; the MMA reads the first 64)
+        const int nb0 = (tile / num_m) * BN +
+                        (half < 0 ? static_cast<int>(rank) * BNH : half * BNH + static_cast<int>(rank) * (BNH / 2));
         for (int kb = 0; kb < kb_all; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.status, p.wait_limit_ns)) break;
           uint8_t* sa = smem + stage * STAGE_BYTES;
@@ -199,12 +233,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (leader only)
     if (leader && lane == 0) {
-      const uint32_t idesc_i = idesc_i8_s32(2 * BM, BN);
-      const uint32_t idesc_f = idesc_f16_f32(2 * BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (int tile = pair; tile < tiles && !*s_abort; tile += npairs, ++it) {
+      for (int u = pair; u < U.units && !*s_abort; u += npairs, ++it) {
+        int tile, half;
+        U.at(u, tile, half);
+        const int nt = half < 0 ? BN : BNH;
+        const uint32_t idesc_i = idesc_i8_s32(2 * BM, nt);
+        const uint32_t idesc_f = idesc_f16_f32(2 * BM, nt);
         const int buf = dbl ? (it & 1) : 0;
         const uint32_t use = dbl ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
         if (!mbar_wait_bounded(&acc_empty[buf], (use & 1u) ^ 1u, s_abort, p.status, p.wait_limit_ns)) break;
@@ -260,9 +297,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint8_t* stg = smem + STG_OFF + ew * 2 * STG_BYTES;
     int stg_i = 0;
     int it = 0;
-    for (int tile = pair; tile < tiles; tile += npairs, ++it) {  // abort is seen by the wait below
+    for (int u = pair; u < U.units; u += npairs, ++it) {  // abort is seen by the wait below
+      int tile, half;
+      U.at(u, tile, half);
       const int row_base = (tile % num_m) * (2 * BM) + static_cast<int>(rank) * BM + quad * 32;
-      const int n0 = (tile / num_m) * BN + col_half * BNH;
+      // whole tile: 128 columns (4 chunks) per warp; half tile: 64 (2 chunks)
+      const int nch = half < 0 ? CHUNKS : CHUNKS / 2;
+      const int col_off = col_half * nch * 32;  // TMEM column of this warp's first chunk
+      const int n0 = (tile / num_m) * BN + (half < 0 ? 0 : half * BNH) + col_off;
       const int buf = dbl ? (it & 1) : 0;
       const uint32_t use = dbl ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
       // Everything this tile needs besides the accumulators is fetched before
@@ -272,7 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int cc = 0; cc < CHUNKS; ++cc) {
         const int n = n0 + cc * 32 + lane;
-        const bool in = !RAW && n < N;
+        const bool in = !RAW && cc < nch && n < N;
         sb_r[cc] = in ? __ldg(p.SCB + n) : 0.f;
         bi_r[cc] = (in && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
       }
@@ -309,7 +351,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int cb = 0; cb < 4; ++cb) {
             const int n = n0 + cc * 32 + cb * 8 + g;
-            if (n < N) {
+            if (cc < nch && n < N) {
               const uint32_t* w = reinterpret_cast<const uint32_t*>(p.WO + static_cast<size_t>(n) * p.ld_o + 2 * tq);
               bf[cc][cb][0] = __ldg(w);
               bf[cc][cb][1] = __ldg(w + 4);
@@ -323,10 +365,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (lane == 0) ok = mbar_wait_bounded(&acc_full[buf], use & 1u, s_abort, p.status, p.wait_limit_ns) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after_sync();
-      const uint32_t t_int = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + col_half * BNH);
-      const uint32_t t_fp = tmem_base + lane_off + static_cast<uint32_t>(BN + col_half * BNH);
+      const uint32_t t_int = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + col_off);
+      const uint32_t t_fp = tmem_base + lane_off + static_cast<uint32_t>(BN + col_off);
 #pragma unroll
       for (int cc = 0; cc < CHUNKS; ++cc) {
+        if (cc >= nch) break;
         uint32_t c[2][16];  // int32 accumulators of row blocks 0 / 1
         tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
         tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
@@ -337,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tmem_wait_ld();
         const int nb = n0 + cc * 32;
-        if (RAW) {
+        if constexpr (RAW) {
 #pragma unroll
           for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
@@ -356,8 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                   if (n + 1 < N) dst[1] = static_cast<int32_t>(v1);
                 }
               }
-          continue;
-        }
+        } else {
         // dequant in fragment layout; halves[rb][cb][hh] = (row rb*16+g+8hh, columns cb*8+2tq, +1)
         uint32_t halves[2][4][2];
 #pragma unroll
@@ -430,6 +472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
               }
         }
+        }  // RAW / fused
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -489,7 +532,8 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, bool raw_int32,
   }
   const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
   const int pairs_fit = max_pairs(raw_int32, num_sms);
-  const int pairs = tiles < pairs_fit ? tiles : pairs_fit;
+  // fewer tiles than pairs: run each tile as two half tiles where that fits
+  const int pairs = tiles >= pairs_fit ? pairs_fit : (2 * tiles <= pairs_fit ? 2 * tiles : tiles);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);

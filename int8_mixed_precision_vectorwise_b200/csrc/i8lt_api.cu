@@ -55,7 +55,8 @@ bool ws_layout(int M, int N, int K, int cap, WsLayout* L) {
   L->wo = off;
   off += L->decode ? 0 : align256(static_cast<size_t>(N) * L->ld_o * 2);
   L->partials = off;
-  off += L->decode ? align256(static_cast<size_t>(i8lt::decode_slots(N, K)) * i8lt::kDecodeMaxTokens * N * 4) : 0;
+  // int32 partials, then fp32 partials of the outlier term
+  off += L->decode ? align256(static_cast<size_t>(i8lt::decode_slots(N, K)) * i8lt::kDecodeMaxTokens * N * 8) : 0;
   L->total = off;
   return true;
 }
@@ -194,7 +195,14 @@ i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int 
   const bool outliers = threshold > 0.f;
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
-  // status word, counts, bitmap and split-K counters are contiguous: one memset clears them
+  if (L.decode) {
+    // one cluster launch writes everything the decode GEMM reads, header and counters included
+    const int n_counters = ((N + 127) / 128) * 4;
+    return cuda_status(i8lt::launch_decode_prep(Xh, M, K, threshold, cap, w.CA, w.SCA, w.idx,
+                                                cap > 0 ? w.XO : nullptr, L.ld_o, w.hdr, w.counters, n_counters,
+                                                st));
+  }
+  // status word, counts and bitmap are contiguous: one memset clears them
   if (cudaMemsetAsync(workspace, 0, L.clear_bytes, st) != cudaSuccess) return I8_ERR_CUDA;
   i8_status s = cuda_status(
       i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr, w.hdr, sms, st));
@@ -219,13 +227,13 @@ i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_ha
     d.SCB = SCB;
     d.bias = reinterpret_cast<const __half*>(bias);
     d.out = reinterpret_cast<__half*>(out);
-    d.CB = CB;
     d.idx = w.idx;
     d.n_used = with_o ? reinterpret_cast<const int32_t*>(w.hdr + 1) : nullptr;
     d.out_cap = cap;
     d.XO = w.XO;
     d.ld_o = L.ld_o;
     d.partials = w.partials;
+    d.slots = i8lt::decode_slots(N, K);
     d.counters = w.counters;
     d.status = w.hdr;
     d.wait_limit_ns = kWaitLimitNs;

@@ -72,13 +72,14 @@ struct DecodeArgs {
   const float* SCB;          // [N]
   const __half* bias;        // [N] or nullptr
   __half* out;               // [M, N]
-  const int8_t* CB;          // [N, K] (outlier columns are read from it directly)
   const int32_t* idx;        // sorted outlier columns
   const int32_t* n_used;     // device count of outlier columns, or nullptr
   int out_cap;
   const __half* XO;          // [M, ld_o] gathered X[:, O]
   int ld_o;
-  int32_t* partials;         // [slots][16][N] split-K partial sums
+  int32_t* partials;         // [slots][16][N] int32 split-K partial sums, then [slots][16][N] fp32
+                             // partial sums of the outlier term
+  int slots;                 // decode_slots(N, K)
   int32_t* counters;         // [ceil(N/128) * 4], zero on entry
   uint32_t* status;
   uint64_t wait_limit_ns;
@@ -96,6 +97,15 @@ inline int decode_slots(int N, int K) {
 // boxes_per_stage: 128-byte K boxes per pipeline stage (1, 2 or 4).
 cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
                                int boxes_per_stage, cudaStream_t st);
+
+// Few-token preparation on one cluster of kDecodePrepCluster CTAs (M <= 16):
+// codes, SCA, outlier list, X_O (zero padded to a multiple of 16 columns), the
+// header words (status, used, total) and zeroed split-K counters, all in one
+// launch.  XO may be null when cap == 0.
+constexpr int kDecodePrepCluster = 8;
+cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA,
+                               int32_t* idx, __half* XO, int ld_o, uint32_t* hdr, int32_t* counters, int n_counters,
+                               cudaStream_t st);
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 

@@ -41,10 +41,15 @@ __device__ __forceinline__ void scan8(const uint4& v, float tau, bool use_tau, f
   }
 }
 
-__device__ __forceinline__ uint32_t code_byte(float x, float r) {
-  int q = __float2int_rn(__fmul_rn(x, r));
-  q = max(-127, min(127, q));
-  return static_cast<uint32_t>(q) & 0xFFu;
+// int8 code of x * r, rounded to nearest even.  The convert saturates to
+// [-128, 127]; that equals clipping to [-127, 127] for every element kept on
+// the int8 path (|x| <= amax, so |x * r| <= 127 * (1 + 2^-23)).  Elements at or
+// above the threshold may saturate to -128, but their columns are outlier
+// columns, whose codes are zeroed before use.
+__device__ __forceinline__ uint32_t code_s8(float x, float r) {
+  uint32_t q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(x, r)));
+  return q;
 }
 
 // 8 fp16 values -> 8 int8 codes packed little-endian.
@@ -55,21 +60,46 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float r) {
   for (int p = 0; p < 2; ++p) {
     const float2 a = __half22float2(h[2 * p]);
     const float2 b = __half22float2(h[2 * p + 1]);
-    w[p] = code_byte(a.x, r) | (code_byte(a.y, r) << 8) | (code_byte(b.x, r) << 16) | (code_byte(b.y, r) << 24);
+    const uint32_t lo = __byte_perm(code_s8(a.x, r), code_s8(a.y, r), 0x0040);
+    const uint32_t hi = __byte_perm(code_s8(b.x, r), code_s8(b.y, r), 0x0040);
+    w[p] = __byte_perm(lo, hi, 0x5410);
   }
   return make_uint2(w[0], w[1]);
 }
 
-// OR a vector's outlier bits into the global bitmap.  Must be called by all 32
-// lanes of a warp whose lanes hold consecutive vectors (vector index vi).
-__device__ __forceinline__ void publish_outliers(uint32_t big, int vi, uint32_t* bitmap) {
-  if (!__any_sync(kFull, big != 0)) return;
-  uint32_t bits = big << ((vi & 3) * 8);
-  bits |= __shfl_xor_sync(kFull, bits, 1);
-  bits |= __shfl_xor_sync(kFull, bits, 2);
-  if ((threadIdx.x & 3) == 0 && bits) {
-    uint32_t* w = bitmap + (vi >> 2);
-    if ((__ldcg(w) & bits) != bits) atomicOr(w, bits);   // skip the atomic once set
+// Max |x| of 8 fp16 values with packed fp16 max (exact: the max of fp16
+// values is one of them).
+__device__ __forceinline__ float absmax8(const uint4& v) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  const __half2 m = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+// Fold one vector into the row's running absmax.  A vector whose max reaches
+// the threshold takes the per-element path: its outliers are left out of the
+// max and OR-ed into the block's shared-memory bitmap (vector vi covers
+// columns 8vi .. 8vi+7, i.e. bits 8(vi % 4) .. of word vi / 4).
+__device__ __forceinline__ void fold8(const uint4& v, int vi, float tau, bool use_tau, float& amax,
+                                      uint32_t* sbm) {
+  const float vmax = absmax8(v);
+  if (!use_tau || vmax < tau) {
+    amax = fmaxf(amax, vmax);
+    return;
+  }
+  uint32_t big = 0;
+  scan8(v, tau, true, amax, big);
+  atomicOr(sbm + (vi >> 2), big << ((vi & 3) * 8));
+}
+
+// The block's outlier bitmap lives in shared memory while its rows are
+// scanned; each non-zero word reaches the global bitmap with one atomic.
+__device__ __forceinline__ void sbm_clear(uint32_t* sbm, int nwords) {
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) sbm[w] = 0u;
+}
+__device__ __forceinline__ void sbm_flush(const uint32_t* sbm, int nwords, uint32_t* bitmap) {
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) {
+    const uint32_t bits = sbm[w];
+    if (bits) atomicOr(bitmap + w, bits);
   }
 }
 
@@ -83,17 +113,17 @@ __global__ void __launch_bounds__(256) k_quant_rows(const __half* __restrict__ X
                                                     int8_t* __restrict__ CA, float* __restrict__ SCA,
                                                     uint32_t* __restrict__ bitmap) {
   static_assert(G % 32 == 0 && 256 % G == 0, "group size");
+  extern __shared__ uint32_t sbm[];
+  __shared__ float red[8];
   pdl_launch_dependents();
   constexpr int ROWS = 256 / G;
   constexpr int WPR = G / 32;  // warps per row
-  __shared__ float red[8];
-
   const int tid = threadIdx.x;
   const int g = tid / G;
   const int t = tid % G;
   const int row = blockIdx.x * ROWS + g;
   const bool valid = row < M;
-  const int nvec = K >> 3;
+  const int nvec = K >> 3, nwords = (K + 31) >> 5;
   const bool use_tau = tau > 0.f;
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(valid ? row : 0) * K);
 
@@ -103,13 +133,13 @@ __global__ void __launch_bounds__(256) k_quant_rows(const __half* __restrict__ X
     const int vi = t + i * G;
     v[i] = (valid && vi < nvec) ? ld_stream_16(xr + vi) : make_uint4(0, 0, 0, 0);
   }
+  if (use_tau) {
+    sbm_clear(sbm, nwords);
+    __syncthreads();
+  }
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    uint32_t big = 0;
-    scan8(v[i], tau, use_tau, amax, big);
-    if (use_tau) publish_outliers(big, t + i * G, bitmap);
-  }
+  for (int i = 0; i < VPT; ++i) fold8(v[i], t + i * G, tau, use_tau, amax, sbm);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
   if constexpr (WPR > 1) {
@@ -129,6 +159,10 @@ __global__ void __launch_bounds__(256) k_quant_rows(const __half* __restrict__ X
       if (vi < nvec) cr[vi] = quant8(v[i], r);
     }
   }
+  if (use_tau) {
+    __syncthreads();
+    sbm_flush(sbm, nwords, bitmap);
+  }
 }
 
 // Rows too long to cache in registers: one block per row, X read twice (the
@@ -136,20 +170,19 @@ __global__ void __launch_bounds__(256) k_quant_rows(const __half* __restrict__ X
 __global__ void __launch_bounds__(256) k_quant_rows_stream(const __half* __restrict__ X, int M, int K,
                                                            float tau, int8_t* __restrict__ CA,
                                                            float* __restrict__ SCA, uint32_t* __restrict__ bitmap) {
+  extern __shared__ uint32_t sbm[];
   __shared__ float red[8];
   pdl_launch_dependents();
   const int row = blockIdx.x;
-  const int nvec = K >> 3;
+  const int nvec = K >> 3, nwords = (K + 31) >> 5;
   const bool use_tau = tau > 0.f;
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * K);
-  float amax = 0.f;
-  for (int base = 0; base < nvec; base += 256) {   // uniform trip count for the warp shuffles
-    const int vi = base + threadIdx.x;
-    const uint4 v = vi < nvec ? xr[vi] : make_uint4(0, 0, 0, 0);
-    uint32_t big = 0;
-    scan8(v, tau, use_tau, amax, big);
-    if (use_tau) publish_outliers(big, vi, bitmap);
+  if (use_tau) {
+    sbm_clear(sbm, nwords);
+    __syncthreads();
   }
+  float amax = 0.f;
+  for (int vi = threadIdx.x; vi < nvec; vi += 256) fold8(xr[vi], vi, tau, use_tau, amax, sbm);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
@@ -161,69 +194,7 @@ __global__ void __launch_bounds__(256) k_quant_rows_stream(const __half* __restr
   if (threadIdx.x == 0) SCA[row] = amax;
   uint2* cr = reinterpret_cast<uint2*>(CA + static_cast<size_t>(row) * K);
   for (int vi = threadIdx.x; vi < nvec; vi += 256) cr[vi] = quant8(xr[vi], r);
-}
-
-// Persistent warp-per-row variant for many rows.  Pass 1 streams the row from
-// HBM, U 16-byte loads per lane in flight, and reduces |x| with packed fp16
-// max (exact: the max of fp16 values is one of them); only vectors whose max
-// reaches the threshold take the per-element fp32 path that separates
-// outliers.  Pass 2 re-reads the row (now in L2) and writes the codes.  No
-// block-level synchronisation: every warp walks its own rows.
-template <int U>
-__global__ void __launch_bounds__(256) k_quant_rows_warp(const __half* __restrict__ X, int M, int K, float tau,
-                                                         int8_t* __restrict__ CA, float* __restrict__ SCA,
-                                                         uint32_t* __restrict__ bitmap) {
-  pdl_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const int nwarps = gridDim.x * (blockDim.x >> 5);
-  const int nvec = K >> 3;
-  const bool use_tau = tau > 0.f;
-  for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < M; row += nwarps) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * K);
-    float amax = 0.f;
-    for (int base = 0; base < nvec; base += 32 * U) {  // uniform trip count for the warp votes
-      uint4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int vi = base + u * 32 + lane;
-        v[u] = vi < nvec ? __ldg(xr + vi) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const __half2* h = reinterpret_cast<const __half2*>(&v[u]);
-        const __half2 m = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
-        const float vmax = fmaxf(__low2float(m), __high2float(m));
-        const bool hot = use_tau && vmax >= tau;  // some element of this vector is an outlier
-        if (__any_sync(kFull, hot)) {
-          uint32_t big = 0;
-          float keep = 0.f;
-          if (hot) scan8(v[u], tau, true, keep, big); else keep = vmax;
-          amax = fmaxf(amax, keep);
-          publish_outliers(big, base + u * 32 + lane, bitmap);
-        } else {
-          amax = fmaxf(amax, vmax);
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-    const float r = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
-    if (lane == 0) SCA[row] = amax;
-    uint2* cr = reinterpret_cast<uint2*>(CA + static_cast<size_t>(row) * K);
-    for (int base = 0; base < nvec; base += 32 * U) {
-      uint4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int vi = base + u * 32 + lane;
-        if (vi < nvec) v[u] = __ldcs(xr + vi);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int vi = base + u * 32 + lane;
-        if (vi < nvec) cr[vi] = quant8(v[u], r);
-      }
-    }
-  }
+  if (use_tau) sbm_flush(sbm, nwords, bitmap);  // the __syncthreads above ordered every mark before this
 }
 
 // Zero every outlier column of CA straight from the bitmap (one warp per row).
@@ -247,8 +218,8 @@ __global__ void __launch_bounds__(256) k_zero_outlier_cols(const uint32_t* __res
 
 // Outlier preparation for the fused forward.  Every block rebuilds the sorted
 // column list from the bitmap in shared memory (a block-wide scan of popcounts),
-// then the grid's warps walk rows: X rows (zero CA[:, O], gather X[:, O]) and
-// CB rows (gather fp16(CB[:, O])).  Gathered rows are zero-padded to a multiple
+// then the grid's threads walk rows, one row each: X rows (zero CA[:, O],
+// gather X[:, O]) and CB rows (gather fp16(CB[:, O])).  Gathered rows are zero-padded to a multiple
 // of 64 columns (one 128-byte fp16 tile).  Block 0 publishes the list, the
 // counts and the overflow status.
 __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restrict__ bitmap, int K, int cap,
@@ -315,22 +286,36 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
   const int n_pad = (used + 63) & ~63;
   const int rows_x = (XO != nullptr || CA != nullptr) ? M : 0;
   const int rows_w = WO != nullptr ? N : 0;
-  const __half zero = __float2half_rn(0.f);
-  for (int r = blockIdx.x * 8 + warp; r < rows_x + rows_w; r += gridDim.x * 8) {
-    if (r < rows_x) {
-      const size_t base = static_cast<size_t>(r) * K;
-      for (int c = lane; c < n_pad; c += 32) {
-        const int j = c < used ? idx_s[c] : -1;
-        if (XO) XO[static_cast<size_t>(r) * ld_o + c] = j >= 0 ? X[base + j] : zero;
-        if (CA && j >= 0) CA[base + j] = 0;
+  // One thread per row: its `used` gathers are independent loads issued
+  // together, then the gathered row (zero padded) leaves as 16-byte stores.
+  for (int r = blockIdx.x * 256 + threadIdx.x; r < rows_x + rows_w; r += gridDim.x * 256) {
+    const bool is_x = r < rows_x;
+    const int row = is_x ? r : r - rows_x;
+    const size_t base = static_cast<size_t>(row) * K;
+    __half* dst = is_x ? (XO != nullptr ? XO + static_cast<size_t>(row) * ld_o : nullptr)
+                       : WO + static_cast<size_t>(row) * ld_o;
+    for (int c0 = 0; c0 < n_pad; c0 += 8) {
+      uint32_t h[4] = {0u, 0u, 0u, 0u};
+      if (c0 < used) {
+        unsigned short v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          v[q] = 0;
+          if (c0 + q < used) {
+            const int j = idx_s[c0 + q];
+            v[q] = is_x ? __half_as_ushort(X[base + j])
+                        : __half_as_ushort(__int2half_rn(static_cast<int>(CB[base + j])));
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) h[q] = static_cast<uint32_t>(v[2 * q]) | (static_cast<uint32_t>(v[2 * q + 1]) << 16);
+        if (is_x && CA != nullptr) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (c0 + q < used) CA[base + idx_s[c0 + q]] = 0;
+        }
       }
-    } else {
-      const int n = r - rows_x;
-      const size_t base = static_cast<size_t>(n) * K;
-      for (int c = lane; c < n_pad; c += 32) {
-        const int j = c < used ? idx_s[c] : -1;
-        WO[static_cast<size_t>(n) * ld_o + c] = j >= 0 ? __int2half_rn(static_cast<int>(CB[base + j])) : zero;
-      }
+      if (dst != nullptr) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(h[0], h[1], h[2], h[3]);
     }
   }
 }
@@ -402,32 +387,23 @@ __global__ void __launch_bounds__(256) k_dequant(const int8_t* __restrict__ CB, 
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
                               uint32_t* status, int num_sms, cudaStream_t st) {
   (void)status;
-  // Many rows: persistent warps, one row each at a time.
-  if (M >= 8 * num_sms) {
-    static int blocks_per_sm = 0;
-    if (blocks_per_sm == 0) {
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, k_quant_rows_warp<8>, 256, 0) !=
-              cudaSuccess ||
-          blocks_per_sm <= 0)
-        blocks_per_sm = 4;
-    }
-    const int warps = (M + 0) < num_sms * blocks_per_sm * 8 ? M : num_sms * blocks_per_sm * 8;
-    k_quant_rows_warp<8><<<(warps + 7) / 8, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
-    return cudaGetLastError();
-  }
+  const size_t smem = tau > 0.f ? static_cast<size_t>((K + 31) / 32) * 4 : 0;
   const int nvec = K / 8;
+  // One row per group of threads with the row in registers (one pass over X),
+  // grids of many small blocks so that enough rows are in flight per SM; rows
+  // beyond 32768 columns stream twice.
   if (nvec <= 32 * 8) {
-    k_quant_rows<32, 8><<<(M + 7) / 8, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
+    k_quant_rows<32, 8><<<(M + 7) / 8, 256, smem, st>>>(X, M, K, tau, CA, SCA, bitmap);
   } else if (nvec <= 64 * 8) {
-    k_quant_rows<64, 8><<<(M + 3) / 4, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
+    k_quant_rows<64, 8><<<(M + 3) / 4, 256, smem, st>>>(X, M, K, tau, CA, SCA, bitmap);
   } else if (nvec <= 128 * 8) {
-    k_quant_rows<128, 8><<<(M + 1) / 2, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
+    k_quant_rows<128, 8><<<(M + 1) / 2, 256, smem, st>>>(X, M, K, tau, CA, SCA, bitmap);
   } else if (nvec <= 256 * 8) {
-    k_quant_rows<256, 8><<<M, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
+    k_quant_rows<256, 8><<<M, 256, smem, st>>>(X, M, K, tau, CA, SCA, bitmap);
   } else if (nvec <= 256 * 16) {
-    k_quant_rows<256, 16><<<M, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
+    k_quant_rows<256, 16><<<M, 256, smem, st>>>(X, M, K, tau, CA, SCA, bitmap);
   } else {
-    k_quant_rows_stream<<<M, 256, 0, st>>>(X, M, K, tau, CA, SCA, bitmap);
+    k_quant_rows_stream<<<M, 256, smem, st>>>(X, M, K, tau, CA, SCA, bitmap);
   }
   return cudaGetLastError();
 }
@@ -444,7 +420,7 @@ cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32
                                    __half* XO, const int8_t* CB, int N, __half* WO, int ld_o, int num_sms,
                                    cudaStream_t st) {
   const int rows = ((XO || CA) ? M : 0) + (WO ? N : 0);
-  const int blocks = max(1, min((rows + 7) / 8, num_sms * 4));
+  const int blocks = max(1, min((rows + 255) / 256, num_sms * 4));
   const size_t smem = static_cast<size_t>(max(cap, 1)) * sizeof(int32_t);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks, 1, 1);

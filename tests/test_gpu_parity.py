@@ -121,8 +121,13 @@ def test_weight_quant_matches_oracle(i8):
 
 
 # ------------------------------------------------------------------ int8 GEMM
+# Tile schedules on 148 SMs (74 CTA pairs, 256 x 256 tiles): up to 37 tiles run
+# as half tiles only; (4096, 4096) and (2048, 5120) end with a round of half
+# tiles; (1792, 4864) and (2304, 4096) leave too many tiles for that and run
+# whole tiles only.
 GSHAPES = [(128, 256, 128), (1, 1, 16), (37, 300, 272), (300, 520, 1040), (256, 512, 4096), (513, 257, 160),
-           (129, 1000, 2064), (16, 4096, 28672), (1024, 768, 512)]
+           (129, 1000, 2064), (16, 4096, 28672), (1024, 768, 512), (4096, 4096, 256), (2048, 5120, 256),
+           (1792, 4864, 128), (2304, 4096, 144)]
 
 
 @pytest.mark.parametrize("M,N,K", GSHAPES)
@@ -197,6 +202,11 @@ FSHAPES = [
     (513, 700, 2048, 70, 6.0, True),     # two fp16 k-blocks of outliers
     (200, 384, 512, 3, 0.0, False),      # threshold 0: outlier columns stay on the int8 path
     (4, 28672, 8192, 8, 6.0, False),     # decode-shaped
+    (3, 300, 272, 3, 6.0, True),         # decode-shaped, K split unevenly over the preparation cluster
+    (16, 2048, 4096, 40, 6.0, True),     # decode-shaped, outliers in every CTA's column range
+    (4096, 4096, 512, 4, 6.0, True),     # whole tiles, then a round of half tiles
+    (2048, 5120, 1024, 70, 6.0, False),  # the same with the fp16 outlier k-blocks
+    (2304, 4096, 256, 5, 6.0, True),     # whole tiles only
 ]
 
 
@@ -208,9 +218,10 @@ def test_linear8bit_forward(i8, M, N, K, n_out, tau, with_bias):
     assert_close(out, ref, "forward")
 
 
-def test_forward_all_columns_outliers(i8):
+@pytest.mark.parametrize("M", [64, 8])
+def test_forward_all_columns_outliers(i8, M):
     """Threshold below every magnitude: the int8 path is empty and out is the fp16 path alone."""
-    M, N, K = 64, 256, 128
+    N, K = 256, 128
     X, _ = act(M, K, 0, seed=3)
     X[0] = np.where(np.abs(X[0]) < 1e-2, np.float16(0.5), X[0])
     out, ref, code, count, n_ref = None, None, None, None, None
@@ -222,8 +233,9 @@ def test_forward_all_columns_outliers(i8):
     assert_close(host(o), oracle.linear8bit_forward(X, rCB, rSCB, None, 1e-3), "all-outlier")
 
 
-def test_forward_outlier_overflow_status(i8):
-    M, N, K = 32, 256, 512
+@pytest.mark.parametrize("M", [32, 4])
+def test_forward_outlier_overflow_status(i8, M):
+    N, K = 256, 512
     X, _ = act(M, K, 20, seed=4)
     W = wl.weight(9, N, K)
     rCB, rSCB = oracle.quantize_weight_rowwise(W)
