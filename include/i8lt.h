@@ -150,10 +150,13 @@ I8_API size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_
  *   workspace / workspace_bytes: see i8_linear8bit_workspace_size.
  *   max_outlier_cols: capacity for |O|; if more columns reach the threshold,
  *   the status word becomes I8_ERR_OUTLIER_OVERFLOW and out is unspecified.
- * Enqueues one small memset and three kernels: the fused quantiser, the
- * outlier preparation (skipped when threshold == 0) and the tensor-core GEMM
- * with the dequant epilogue.  Identical to i8_linear8bit_prepare followed by
- * i8_linear8bit_matmul_dequant on the same stream and workspace.
+ * For M > 16 it enqueues one small memset and three kernels: the fused
+ * quantiser, the outlier preparation (skipped when threshold == 0) and the
+ * tensor-core GEMM with the dequant epilogue.  For M <= 16 it enqueues two
+ * kernels: one cluster launch that does the quantisation and the outlier
+ * preparation (and writes the status word itself), and the few-token GEMM.
+ * Identical to i8_linear8bit_prepare followed by i8_linear8bit_matmul_dequant
+ * on the same stream and workspace.
  */
 I8_API i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const float* SCB,
                                 const i8_half* bias, int M, int N, int K, float threshold,
@@ -163,10 +166,10 @@ I8_API i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const
 /*
  * The two halves of i8_linear8bit_forward, for callers that want to place
  * work or events between them (same arguments, same workspace, same stream):
- *   i8_linear8bit_prepare: clears the status word and bitmap, quantises X into
- *     the workspace (CA, SCA, outlier bitmap) and, when threshold > 0, builds
- *     the outlier column list, zeroes CA's outlier columns and gathers the fp16
- *     operands X[:, O] and CB[:, O].
+ *   i8_linear8bit_prepare: resets the status word, quantises X into the
+ *     workspace (CA, SCA) and, when threshold > 0, finds the outlier columns,
+ *     builds their sorted list, zeroes CA's outlier columns and gathers the
+ *     fp16 operands X[:, O] (and, for M > 16, CB[:, O]).
  *   i8_linear8bit_matmul_dequant: the tensor-core GEMM with the fused
  *     dequant / bias / outlier epilogue, reading the prepared workspace.
  *     Enqueue it right after i8_linear8bit_prepare on the same stream (events
