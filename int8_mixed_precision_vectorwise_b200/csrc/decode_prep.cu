@@ -33,6 +33,8 @@ namespace {
 constexpr int PC = kDecodePrepCluster;   // CTAs in the cluster
 constexpr int PT = 1024;                 // threads per CTA
 constexpr unsigned kAll = 0xffffffffu;
+constexpr int PU = 8;                    // X vectors per thread in flight
+constexpr int kLocalList = 1024;         // outlier columns per CTA gathered in parallel
 
 __device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t cluster_addr) {
   uint32_t v;
@@ -57,6 +59,7 @@ __global__ void __cluster_dims__(kDecodePrepCluster, 1, 1) __launch_bounds__(102
   __shared__ int s_count, s_before, s_total;
   __shared__ int s_warp[PT / 32];
   __shared__ float s_r[kDecodeMaxTokens];
+  __shared__ int s_list[kLocalList];     // this CTA's outlier columns, in list order
 
   pdl_launch_dependents();  // the GEMM may be scheduled now; it waits for this grid before reading
   pdl_wait();               // X and the workspace may belong to the work queued before
@@ -76,35 +79,51 @@ __global__ void __cluster_dims__(kDecodePrepCluster, 1, 1) __launch_bounds__(102
   __syncthreads();
 
   // ---------------------------------------------------------------- pass 1
-  for (int base = 0; base < items; base += PT) {  // uniform trip count: whole warps vote below
-    const int it = base + tid;
-    const bool valid = it < items;
-    const int r = valid ? it / nv : -1;
-    float keep = 0.f;
-    if (valid) {
-      const int v = it - r * nv;
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + c0) + v);
-      const __half2* h = reinterpret_cast<const __half2*>(&x);
-      const __half2 m = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
-      const float vmax = fmaxf(__low2float(m), __high2float(m));
-      if (!use_tau || vmax < tau) {
-        keep = vmax;
-      } else {
-        uint32_t big = 0;
+  // Items (row, 8-column vector) in chunks of PU per thread: all PU loads are
+  // issued before any is used.  When the CTA's part of X fits in one chunk it
+  // stays in registers for pass 2.
+  uint4 xv[PU];
+  const bool one_chunk = items <= PU * PT;
+  for (int base = 0; base < items; base += PU * PT) {  // uniform trip count: whole warps vote below
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(h[e]);
-          const float a0 = fabsf(f.x), a1 = fabsf(f.y);
-          if (a0 >= tau) big |= 1u << (2 * e); else keep = fmaxf(keep, a0);
-          if (a1 >= tau) big |= 2u << (2 * e); else keep = fmaxf(keep, a1);
-        }
-        atomicOr(s_flags + (v >> 2), big << ((v & 3) * 8));
+    for (int u = 0; u < PU; ++u) {
+      const int it = base + u * PT + tid;
+      xv[u] = make_uint4(0, 0, 0, 0);
+      if (it < items) {
+        const int r = it / nv;
+        xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + c0) + (it - r * nv));
       }
     }
-    // lanes of the same row combine their maxima; one shared atomic per row and warp
-    const unsigned same = __match_any_sync(kAll, r);
-    const unsigned mx = __reduce_max_sync(same, __float_as_uint(keep));
-    if (valid && lane == __ffs(same) - 1) atomicMax(s_rowmax + r, mx);
+#pragma unroll
+    for (int u = 0; u < PU; ++u) {
+      const int it = base + u * PT + tid;
+      const bool valid = it < items;
+      const int r = valid ? it / nv : -1;
+      float keep = 0.f;
+      if (valid) {
+        const int v = it - r * nv;
+        const __half2* h = reinterpret_cast<const __half2*>(&xv[u]);
+        const __half2 m = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
+        const float vmax = fmaxf(__low2float(m), __high2float(m));
+        if (!use_tau || vmax < tau) {
+          keep = vmax;
+        } else {
+          uint32_t big = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            const float a0 = fabsf(f.x), a1 = fabsf(f.y);
+            if (a0 >= tau) big |= 1u << (2 * e); else keep = fmaxf(keep, a0);
+            if (a1 >= tau) big |= 2u << (2 * e); else keep = fmaxf(keep, a1);
+          }
+          atomicOr(s_flags + (v >> 2), big << ((v & 3) * 8));
+        }
+      }
+      // lanes of the same row combine their maxima; one shared atomic per row and warp
+      const unsigned same = __match_any_sync(kAll, r);
+      const unsigned mx = __reduce_max_sync(same, __float_as_uint(keep));
+      if (valid && lane == __ffs(same) - 1) atomicMax(s_rowmax + r, mx);
+    }
   }
   __syncthreads();
   int cnt = 0;
@@ -143,27 +162,41 @@ __global__ void __cluster_dims__(kDecodePrepCluster, 1, 1) __launch_bounds__(102
   const int used = min(total, cap);
 
   // ---------------------------------------------------------------- pass 2: codes
-  for (int it = tid; it < items; it += PT) {
-    const int r = it / nv, v = it - r * nv;
-    const uint4 x = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + c0) + v);
-    const float rs = s_r[r];
-    const uint32_t fl = (s_flags[v >> 2] >> ((v & 3) * 8)) & 0xffu;
-    const __half2* h = reinterpret_cast<const __half2*>(&x);
-    uint32_t w[2];
+  for (int base = 0; base < items; base += PU * PT) {
+    if (!one_chunk) {  // X was too large to keep: read the chunk again (from L2)
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      const float2 a = __half22float2(h[2 * p]);
-      const float2 b = __half22float2(h[2 * p + 1]);
-      const uint32_t lo = __byte_perm(code_s8p(a.x, rs), code_s8p(a.y, rs), 0x0040);
-      const uint32_t hi = __byte_perm(code_s8p(b.x, rs), code_s8p(b.y, rs), 0x0040);
-      w[p] = __byte_perm(lo, hi, 0x5410);
+      for (int u = 0; u < PU; ++u) {
+        const int it = base + u * PT + tid;
+        if (it < items) {
+          const int r = it / nv;
+          xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + c0) + (it - r * nv));
+        }
+      }
     }
-    if (fl) {  // outlier columns carry code 0
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (fl & (1u << e)) w[e >> 2] &= ~(0xffu << ((e & 3) * 8));
+    for (int u = 0; u < PU; ++u) {
+      const int it = base + u * PT + tid;
+      if (it >= items) break;
+      const int r = it / nv, v = it - r * nv;
+      const float rs = s_r[r];
+      const uint32_t fl = (s_flags[v >> 2] >> ((v & 3) * 8)) & 0xffu;
+      const __half2* h = reinterpret_cast<const __half2*>(&xv[u]);
+      uint32_t w[2];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float2 a = __half22float2(h[2 * p]);
+        const float2 b = __half22float2(h[2 * p + 1]);
+        const uint32_t lo = __byte_perm(code_s8p(a.x, rs), code_s8p(a.y, rs), 0x0040);
+        const uint32_t hi = __byte_perm(code_s8p(b.x, rs), code_s8p(b.y, rs), 0x0040);
+        w[p] = __byte_perm(lo, hi, 0x5410);
+      }
+      if (fl) {  // outlier columns carry code 0
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (fl & (1u << e)) w[e >> 2] &= ~(0xffu << ((e & 3) * 8));
+      }
+      *reinterpret_cast<uint2*>(CA + static_cast<size_t>(r) * K + c0 + 8 * v) = make_uint2(w[0], w[1]);
     }
-    *reinterpret_cast<uint2*>(CA + static_cast<size_t>(r) * K + c0 + 8 * v) = make_uint2(w[0], w[1]);
   }
 
   // ---------------------------------------------------------------- outlier list and X_O
@@ -197,10 +230,21 @@ __global__ void __cluster_dims__(kDecodePrepCluster, 1, 1) __launch_bounds__(102
         const int col = c0 + 32 * w + b;
         if (pos < cap) {
           idx[pos] = col;
-          for (int r = 0; r < M; ++r) XO[static_cast<size_t>(r) * ld_o + pos] = X[static_cast<size_t>(r) * K + col];
+          if (pos - before < kLocalList) {
+            s_list[pos - before] = col;  // gathered below by the whole CTA
+          } else {
+            for (int r = 0; r < M; ++r) XO[static_cast<size_t>(r) * ld_o + pos] = X[static_cast<size_t>(r) * K + col];
+          }
         }
         ++pos;
       }
+    }
+    __syncthreads();
+    // X_O for the first kLocalList outlier columns of this CTA: one element per thread
+    const int nl = min(min(s_count, kLocalList), max(cap - before, 0));
+    for (int e = tid; e < nl * M; e += PT) {
+      const int r = e / nl, i = e - r * nl;
+      XO[static_cast<size_t>(r) * ld_o + before + i] = X[static_cast<size_t>(r) * K + s_list[i]];
     }
   }
   if (rank == 0) {
