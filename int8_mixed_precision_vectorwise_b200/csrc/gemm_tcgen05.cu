@@ -307,17 +307,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int n0 = (tile / num_m) * BN + (half < 0 ? 0 : half * BNH) + col_off;
       const int buf = dbl ? (it & 1) : 0;
       const uint32_t use = dbl ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
-      // Everything this tile needs besides the accumulators is fetched before
-      // the accumulator wait, so its latency hides behind the mainloop.
-      // Column scales / bias: lane j holds column cc*32 + j of chunk cc.
-      float sb_r[CHUNKS], bi_r[CHUNKS];
-#pragma unroll
-      for (int cc = 0; cc < CHUNKS; ++cc) {
-        const int n = n0 + cc * 32 + lane;
-        const bool in = !RAW && cc < nch && n < N;
-        sb_r[cc] = in ? __ldg(p.SCB + n) : 0.f;
-        bi_r[cc] = (in && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
-      }
+      // The chunk loop below is deliberately not unrolled: the epilogue runs
+      // beside the TMA and MMA warps, and a compact loop keeps their
+      // instructions resident in the instruction cache.  Data a chunk needs
+      // besides its accumulators is fetched one chunk ahead (the first chunk's
+      // before the accumulator wait).
       // Row scales of this thread's four rows: row_base + g + 8i.
       float sa4[4];
 #pragma unroll
@@ -325,40 +319,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int r = row_base + g + 8 * i;
         sa4[i] = (!RAW && r < M) ? __ldg(p.SCA + r) * (1.0f / 16129.0f) : 0.f;
       }
-      // Few outliers: A fragments (X[:, O] rows) and B fragments (CB[:, O]
-      // columns of the four chunks) of the 16-wide outlier product.
-      uint32_t af[2][4], bf[CHUNKS][4][2];
+      // Few outliers: the A fragments (X[:, O] rows) of the 16-wide outlier
+      // product.  The gathered operands store each group of 16 outlier columns
+      // in the order (0 1 8 9)(2 3 10 11)(4 5 12 13)(6 7 14 15): the four
+      // values a thread needs from a row (columns 2tq, 2tq+1, 2tq+8, 2tq+9)
+      // are one 8-byte load.
+      uint32_t af[2][4];
 #pragma unroll
       for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
         for (int e = 0; e < 4; ++e) af[rb][e] = 0u;
-#pragma unroll
-      for (int cc = 0; cc < CHUNKS; ++cc)
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) bf[cc][cb][0] = bf[cc][cb][1] = 0u;
       if (small_o) {
 #pragma unroll
         for (int rb = 0; rb < 2; ++rb) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = row_base + rb * 16 + g + 8 * (e & 1);
-            const int k = 2 * tq + 8 * (e >> 1);
-            if (r < M) af[rb][e] = __ldg(reinterpret_cast<const uint32_t*>(p.XO + static_cast<size_t>(r) * p.ld_o + k));
-          }
-        }
-#pragma unroll
-        for (int cc = 0; cc < CHUNKS; ++cc) {
-#pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
-            const int n = n0 + cc * 32 + cb * 8 + g;
-            if (cc < nch && n < N) {
-              const uint32_t* w = reinterpret_cast<const uint32_t*>(p.WO + static_cast<size_t>(n) * p.ld_o + 2 * tq);
-              bf[cc][cb][0] = __ldg(w);
-              bf[cc][cb][1] = __ldg(w + 4);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = row_base + rb * 16 + g + 8 * hh;
+            if (r < M) {
+              const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.XO + static_cast<size_t>(r) * p.ld_o + 4 * tq));
+              af[rb][hh] = v.x;
+              af[rb][2 + hh] = v.y;
             }
           }
         }
       }
+      // Per chunk: column scale and bias (lane j holds column nb + j) and the
+      // B fragments (CB[:, O] of the chunk's 32 columns).
+      float sb_n = 0.f, bi_n = 0.f;
+      uint32_t bf_n[4][2];
+      auto fetch_chunk = [&](int cc) {
+        const int n = n0 + cc * 32 + lane;
+        const bool in = !RAW && n < N;
+        sb_n = in ? __ldg(p.SCB + n) : 0.f;
+        bi_n = (in && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+          bf_n[cb][0] = bf_n[cb][1] = 0u;
+          const int nf = n0 + cc * 32 + cb * 8 + g;
+          if (small_o && nf < N) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.WO + static_cast<size_t>(nf) * p.ld_o + 4 * tq));
+            bf_n[cb][0] = v.x;
+            bf_n[cb][1] = v.y;
+          }
+        }
+      };
+      fetch_chunk(0);
       // lane 0 waits for the whole warp, so the warp leaves the loop as one
       // (the TMEM loads below are warp-collective)
       int ok = 0;
@@ -367,9 +372,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tc_fence_after_sync();
       const uint32_t t_int = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + col_off);
       const uint32_t t_fp = tmem_base + lane_off + static_cast<uint32_t>(BN + col_off);
+#pragma unroll 1
+      for (int cc = 0; cc < nch; ++cc) {
+        const float sb_c = sb_n, bi_c = bi_n;
+        uint32_t bf_c[4][2];
 #pragma unroll
-      for (int cc = 0; cc < CHUNKS; ++cc) {
-        if (cc >= nch) break;
+        for (int cb = 0; cb < 4; ++cb) {
+          bf_c[cb][0] = bf_n[cb][0];
+          bf_c[cb][1] = bf_n[cb][1];
+        }
+        if (cc + 1 < nch) fetch_chunk(cc + 1);
         uint32_t c[2][16];  // int32 accumulators of row blocks 0 / 1
         tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
         tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
@@ -405,15 +417,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           const int j = cb * 8 + 2 * tq;
-          const float sb0 = __shfl_sync(0xffffffffu, sb_r[cc], j);
-          const float sb1 = __shfl_sync(0xffffffffu, sb_r[cc], j + 1);
-          const float b0 = __shfl_sync(0xffffffffu, bi_r[cc], j);
-          const float b1 = __shfl_sync(0xffffffffu, bi_r[cc], j + 1);
+          const float sb0 = __shfl_sync(0xffffffffu, sb_c, j);
+          const float sb1 = __shfl_sync(0xffffffffu, sb_c, j + 1);
+          const float b0 = __shfl_sync(0xffffffffu, bi_c, j);
+          const float b1 = __shfl_sync(0xffffffffu, bi_c, j + 1);
 #pragma unroll
           for (int rb = 0; rb < 2; ++rb) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             if (small_o) {
-              mma_16x8x16_f16(d, af[rb], bf[cc][cb][0], bf[cc][cb][1]);
+              mma_16x8x16_f16(d, af[rb], bf_c[cb][0], bf_c[cb][1]);
             } else if (kb_out > 0) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) d[e] = __uint_as_float(f[rb][4 * cb + e]);
@@ -439,11 +451,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-              const int r = rb * 16 + g + 8 * hh;
-#pragma unroll
-              for (int cb = 0; cb < 4; ++cb)
-                *reinterpret_cast<uint32_t*>(box + r * 64 + ((cb ^ ((r >> 1) & 3)) << 4) + 4 * tq) =
-                    halves[rb][cb][hh];
+              // the four 8x8 blocks of rows rb*16 + 8hh .. +7 (one per cb), in the
+              // fragment layout; lane l gives the address of row l % 8 of block l / 8
+              const int blk = lane >> 3, rr = rb * 16 + 8 * hh + (lane & 7);
+              stmatrix_x4(smem_addr(box + rr * 64 + ((blk ^ ((rr >> 1) & 3)) << 4)), halves[rb][0][hh],
+                          halves[rb][1][hh], halves[rb][2][hh], halves[rb][3][hh]);
             }
           fence_async_shared();
           __syncwarp();

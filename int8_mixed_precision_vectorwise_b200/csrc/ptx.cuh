@@ -287,6 +287,15 @@ __device__ __forceinline__ void tma_store_wait_all() {
 }
 
 // Make generic-proxy shared-memory writes visible to the async (TMA) proxy.
+// Four 8x8 16-bit blocks from the mma fragment layout (register j: this
+// thread's two elements of block j) to shared memory; lane l gives the address
+// of row l % 8 of block l / 8.
+__device__ __forceinline__ void stmatrix_x4(uint32_t row_addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(row_addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
+
 __device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ------------------------------------------------------------------ tcgen05, CTA pairs

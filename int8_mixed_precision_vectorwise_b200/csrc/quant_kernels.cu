@@ -109,7 +109,7 @@ __device__ __forceinline__ void sbm_flush(const uint32_t* sbm, int nwords, uint3
 // each thread caching up to VPT 16-byte vectors of its row in registers so X
 // is read from HBM exactly once.
 template <int G, int VPT>
-__global__ void __launch_bounds__(256) k_quant_rows(const __half* __restrict__ X, int M, int K, float tau,
+__global__ void __launch_bounds__(256, (VPT > 8 ? 1 : 5)) k_quant_rows(const __half* __restrict__ X, int M, int K, float tau,
                                                     int8_t* __restrict__ CA, float* __restrict__ SCA,
                                                     uint32_t* __restrict__ bitmap) {
   static_assert(G % 32 == 0 && 256 % G == 0, "group size");
@@ -216,6 +216,17 @@ __global__ void __launch_bounds__(256) k_zero_outlier_cols(const uint32_t* __res
   }
 }
 
+// Position -> list entry of the gathered outlier operands: within each group
+// of 16 columns the entries are stored as (0 1 8 9)(2 3 10 11)(4 5 12 13)
+// (6 7 14 15), so a thread of an m16n8k16 fragment reads its four values
+// (2t, 2t+1, 2t+8, 2t+9) with one 8-byte load.  A product over the outlier
+// columns does not depend on their order, so the tensor-core path that reads
+// whole 64-column tiles uses the same layout.
+__device__ __forceinline__ int outlier_slot(int pos) {
+  const int q = pos & 15;
+  return (pos & ~15) + 2 * (q >> 2) + (q & 1) + 8 * ((q >> 1) & 1);
+}
+
 // Outlier preparation for the fused forward.  Every block rebuilds the sorted
 // column list from the bitmap in shared memory (a block-wide scan of popcounts),
 // then the grid's threads walk rows, one row each: X rows (zero CA[:, O],
@@ -296,13 +307,15 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
                        : WO + static_cast<size_t>(row) * ld_o;
     for (int c0 = 0; c0 < n_pad; c0 += 8) {
       uint32_t h[4] = {0u, 0u, 0u, 0u};
-      if (c0 < used) {
+      if ((c0 & ~15) < used) {  // the 16-column group holds list entries
         unsigned short v[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
+          // stored position c0 + q holds list entry outlier_slot(c0 + q)
+          const int c = outlier_slot(c0 + q);
           v[q] = 0;
-          if (c0 + q < used) {
-            const int j = idx_s[c0 + q];
+          if (c < used) {
+            const int j = idx_s[c];
             v[q] = is_x ? __half_as_ushort(X[base + j])
                         : __half_as_ushort(__int2half_rn(static_cast<int>(CB[base + j])));
           }
@@ -312,7 +325,7 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
         if (is_x && CA != nullptr) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            if (c0 + q < used) CA[base + idx_s[c0 + q]] = 0;
+            if (c0 + q < used) CA[base + idx_s[c0 + q]] = 0;  // every listed column, in list order
         }
       }
       if (dst != nullptr) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(h[0], h[1], h[2], h[3]);

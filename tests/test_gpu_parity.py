@@ -202,6 +202,9 @@ FSHAPES = [
     (513, 700, 2048, 70, 6.0, True),     # two fp16 k-blocks of outliers
     (200, 384, 512, 3, 0.0, False),      # threshold 0: outlier columns stay on the int8 path
     (4, 28672, 8192, 8, 6.0, False),     # decode-shaped
+    (300, 520, 1040, 7, 6.0, True),      # outlier operands: a partly filled 16-column group
+    (256, 512, 2048, 13, 6.0, False),
+    (257, 384, 1024, 17, 6.0, True),     # just past the warp-MMA limit: tensor-core outlier k-block
     (3, 300, 272, 3, 6.0, True),         # decode-shaped, K split unevenly over the preparation cluster
     (16, 2048, 4096, 40, 6.0, True),     # decode-shaped, outliers in every CTA's column range
     (4096, 4096, 512, 4, 6.0, True),     # whole tiles, then a round of half tiles
