@@ -221,6 +221,14 @@ def test_linear8bit_forward(i8, M, N, K, n_out, tau, with_bias):
     assert_close(out, ref, "forward")
 
 
+@pytest.mark.parametrize("n_out", [5, 70])
+def test_forward_large_capacity(i8, n_out):
+    """A capacity above the default 256 (larger list and gathered-operand buffers)."""
+    out, ref, code, count, n_ref = _forward_case(i8, 300, 520, 1040, n_out, 6.0, True, cap=512)
+    assert code == 0 and count == n_ref
+    assert_close(out, ref, "forward (capacity 512)")
+
+
 @pytest.mark.parametrize("M", [64, 8])
 def test_forward_all_columns_outliers(i8, M):
     """Threshold below every magnitude: the int8 path is empty and out is the fp16 path alone."""
