@@ -365,21 +365,51 @@ def run_ours(args):
             h_in.append(None if d.get("chained") else torch.from_numpy(d["X_host"]).pin_memory())
         h_out = [torch.empty(d["out"].shape, dtype=torch.float16).pin_memory() for d in layers]
         Ke = min(K, 20)
+        # Copies run on their own streams so that the host-to-device copy of the
+        # next linear's input and the device-to-host copy of the previous
+        # output (the two directions of the link) overlap the forward: the
+        # forward of linear i waits for its input; the copy of an output waits
+        # for its forward; a forward that rewrites `out` waits for the copy of
+        # its previous contents; a copy that rewrites `X` waits for the forward
+        # that read its previous contents.
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in layers]
+        ev_fwd = [torch.cuda.Event() for _ in layers]
+        ev_out = [torch.cuda.Event() for _ in layers]
+        started = [False] * len(layers)
 
         def e2e_step():
             for li, d in enumerate(layers):
                 L = d["L"]
                 if h_in[li] is not None:
-                    d["X"].copy_(h_in[li], non_blocking=True)
+                    with torch.cuda.stream(s_in):
+                        if started[li]:
+                            s_in.wait_event(ev_fwd[li])
+                        d["X"].copy_(h_in[li], non_blocking=True)
+                        ev_in[li].record(s_in)
+                    st.wait_event(ev_in[li])
+                if started[li]:
+                    st.wait_event(ev_out[li])
                 i8.i8_linear8bit_forward(d["X"], d["CB"], d["SCB"], d["b"], L.threshold, out=d["out"],
                                          workspace=d["ws"], max_outlier_cols=MAX_OUTLIER_COLS)
-                h_out[li].copy_(d["out"], non_blocking=True)
+                ev_fwd[li].record(st)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_fwd[li])
+                    h_out[li].copy_(d["out"], non_blocking=True)
+                    ev_out[li].record(s_out)
+                started[li] = True
+
+        def join():
+            for li in range(len(layers)):
+                st.wait_event(ev_out[li])
         e2e_step()
+        join()
         barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(st)
         for _ in range(Ke):
             e2e_step()
+        join()
         f1.record(st)
         barrier()
         te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)

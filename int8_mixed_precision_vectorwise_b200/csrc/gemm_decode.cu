@@ -47,6 +47,8 @@ constexpr uint32_t DTMEM_COLS = 32;        // two 16-column accumulators
 
 // C boxes (C x 128 bytes of K) per pipeline stage, DRING bytes of ring.
 constexpr int DS_BYTES = DT * DM * 4;      // one segment's outlier term, fp32 [token][row]
+constexpr int XS_COLS = 32;                // outlier columns of X[:, O] kept in shared memory
+constexpr int XS_BYTES = DT * XS_COLS * 2; // fp16 [column][token]
 
 template <int C>
 struct DecodeCfg {
@@ -55,7 +57,8 @@ struct DecodeCfg {
   static constexpr int NUM_BARS = 2 * STAGES + 7;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int DS_OFF = BAR_OFF + ((NUM_BARS * 8 + 15) / 16) * 16;
-  static constexpr int MISC_OFF = DS_OFF + DS_BYTES;
+  static constexpr int XS_OFF = DS_OFF + DS_BYTES;
+  static constexpr int MISC_OFF = XS_OFF + XS_BYTES;
   static constexpr int SMEM_ALLOC = MISC_OFF + 16 + 1024;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
@@ -100,6 +103,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   uint64_t* d_full = mma_done + 1;       // the outlier term of a segment is in d_s
   uint64_t* d_empty = d_full + 1;        // ... and has been read by the 4 epilogue warps
   float* d_s = reinterpret_cast<float*>(smem + Cfg::DS_OFF);
+  __half* x_s = reinterpret_cast<__half*>(smem + Cfg::XS_OFF);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Cfg::MISC_OFF);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -244,6 +248,13 @@ __global__ void __launch_bounds__(DTHREADS, 1)
     // is handed to the epilogue through d_s at the segment's end.
     pdl_wait();  // outlier list and gathered X come from the preceding kernel
     const int n_used = p.n_used != nullptr ? min(max(*p.n_used, 0), p.out_cap) : 0;
+    // the first XS_COLS outlier columns of X, as [column][token], so the
+    // per-stage updates read shared memory instead of waiting on global loads
+    for (int e = lane; e < min(n_used, XS_COLS) * DT; e += 32) {
+      const int j = e / DT, t = e - j * DT;
+      x_s[e] = t < T ? p.XO[static_cast<size_t>(t) * p.ld_o + j] : __float2half_rn(0.f);
+    }
+    __syncwarp();
     int stage = 0;
     uint32_t phase = 0;
     int segi = 0;
@@ -274,7 +285,9 @@ __global__ void __launch_bounds__(DTHREADS, 1)
           const int box = kk >> 7, b = kk & 127;     // 128-byte box, byte within the row
           float x[DT];
 #pragma unroll
-          for (int t = 0; t < DT; ++t) x[t] = t < T ? __half2float(p.XO[static_cast<size_t>(t) * p.ld_o + cur]) : 0.f;
+          for (int t = 0; t < DT; ++t)
+            x[t] = cur < XS_COLS ? __half2float(x_s[cur * DT + t])
+                                 : (t < T ? __half2float(p.XO[static_cast<size_t>(t) * p.ld_o + cur]) : 0.f);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int r = lane + 32 * i;             // 128B swizzle: 16-byte chunk q of row r sits at q ^ (r % 8)

@@ -303,3 +303,30 @@ def test_selftest_bounded_wait_times_out(i8):
     assert time.time() - t0 < 10
     assert int(st.item()) == 5   # I8_ERR_TIMEOUT, and the context is still usable:
     assert torch.ones(4, device="cuda").sum().item() == 4
+
+
+# ------------------------------------------------------------------ CUDA graph capture
+@pytest.mark.parametrize("M,N,K,n_out", [(256, 512, 1024, 3), (4, 4096, 8192, 5)])
+def test_forward_cuda_graph_replay(i8, M, N, K, n_out):
+    """The forward never waits for the host: it can be captured once and replayed on new
+    inputs (a different outlier set each time), the outlier columns being found on the device."""
+    X1, _ = act(M, K, n_out, seed=21)
+    X2, _ = act(M, K, n_out + 2, seed=22)
+    W = wl.weight(23, N, K)
+    b = wl.bias(24, N)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    dX, dCB, dSCB, db = dev(X1), dev(rCB), dev(rSCB), dev(b)
+    out = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    ws = torch.empty((i8.i8_linear8bit_workspace_size(M, N, K, 256),), dtype=torch.uint8, device="cuda")
+    i8.i8_linear8bit_forward(dX, dCB, dSCB, db, 6.0, out=out, workspace=ws)  # first call outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        i8.i8_linear8bit_forward(dX, dCB, dSCB, db, 6.0, out=out, workspace=ws)
+    for X in (X2, X1):
+        dX.copy_(torch.from_numpy(X).cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        _, _, cols = oracle.quantize_rowwise(X, 6.0)
+        assert i8.i8_read_status(ws) == (0, len(cols))
+        assert_close(host(out), oracle.linear8bit_forward(X, rCB, rSCB, b, 6.0), "graph replay")
