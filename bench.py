@@ -144,6 +144,23 @@ class ClockSampler:
                 "sm_mhz_min": min(mhz)}
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+def max_over_ranks(x: float, world: int, dist, device) -> float:
+    """The largest x over all ranks: a job's time is its slowest rank's time."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(ops_per_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job TOPS: every rank (a replica) runs `steps` steps of `ops_per_step`
+    operations; the job takes `ms`, the time of its slowest rank."""
+    return world * ops_per_step * steps / (ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def cpu_oracle_steps(layers_np, rows: int, steps: int, min_seconds: float = 0.0):
     """Run the oracle forward on the first `rows` rows of every linear; returns (seconds per step, ops per step)."""
@@ -352,10 +369,7 @@ def run_ours(args):
     ms = e0.elapsed_time(e1)
     ms_instr = g0.elapsed_time(g1)
     gemm_ms = sum(a.elapsed_time(b) for row in ev for a, b in row)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dist, dev)
 
     # ---- end to end: host inputs -> device -> forward -> host outputs, per step
     e2e = None
@@ -412,14 +426,12 @@ def run_ours(args):
         join()
         f1.record(st)
         barrier()
-        te = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te = max_over_ranks(f0.elapsed_time(f1), world, dist, dev)
         h2d = sum(h.numel() * 2 for h in h_in if h is not None)
         d2h = sum(h.numel() * 2 for h in h_out)
-        e2e = {"value": world * ops_per_step * Ke / (float(te.item()) / 1e3) / 1e12, "unit": "TOPS",
+        e2e = {"value": job_throughput(ops_per_step, Ke, world, te), "unit": "TOPS",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
-               "ms_per_step": float(te.item()) / Ke}
+               "ms_per_step": te / Ke}
 
     for d in layers:
         code, _ = i8.i8_read_status(d["ws"])
@@ -466,7 +478,7 @@ def run_ours(args):
     achieved = ops_per_step * K / (gemm_ms / 1e3) / 1e12
     line = {
         "metric": METRIC,
-        "value": world * ops_per_step * K / (ms_max / 1e3) / 1e12,
+        "value": job_throughput(ops_per_step, K, world, ms_max),
         "unit": "TOPS",
         "n_gpus": world,
         "steps": K,
