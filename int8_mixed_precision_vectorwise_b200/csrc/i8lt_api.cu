@@ -205,7 +205,7 @@ i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int 
   // status word, counts and bitmap are contiguous: one memset clears them
   if (cudaMemsetAsync(workspace, 0, L.clear_bytes, st) != cudaSuccess) return I8_ERR_CUDA;
   i8_status s = cuda_status(
-      i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr, w.hdr, sms, st));
+      i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr, st));
   if (s != I8_OK || !outliers) return s;
   return cuda_status(i8lt::launch_outlier_prepare(w.bitmap, K, cap, reinterpret_cast<int32_t*>(w.hdr + 2),
                                                   reinterpret_cast<int32_t*>(w.hdr + 1), w.idx, w.hdr, w.CA, Xh, M,
@@ -329,7 +329,7 @@ i8_status i8_quantize_rowwise(const i8_half* X, int M, int K, float threshold, i
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
   i8_status s = cuda_status(
-      i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, threshold > 0.f ? bitmap : nullptr, nullptr, sms, st));
+      i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, threshold > 0.f ? bitmap : nullptr, st));
   if (s != I8_OK || threshold == 0.f) return s;
   return cuda_status(i8lt::launch_zero_outlier_cols(bitmap, M, K, CA, sms, st));
 }

@@ -9,9 +9,9 @@
 
 namespace i8lt {
 
-// status: device status word for a pipeline timeout, or nullptr.
+// bitmap: zeroed outlier bitmap to OR into (required when tau > 0).
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
-                              uint32_t* status, int num_sms, cudaStream_t st);
+                              cudaStream_t st);
 cudaError_t launch_zero_outlier_cols(const uint32_t* bitmap, int M, int K, int8_t* CA, int num_sms,
                                      cudaStream_t st);
 cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32_t* total_out, int32_t* used_out,

@@ -398,8 +398,7 @@ __global__ void __launch_bounds__(256) k_dequant(const int8_t* __restrict__ CB, 
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
-                              uint32_t* status, int num_sms, cudaStream_t st) {
-  (void)status;
+                              cudaStream_t st) {
   const size_t smem = tau > 0.f ? static_cast<size_t>((K + 31) / 32) * 4 : 0;
   const int nvec = K / 8;
   // One row per group of threads with the row in registers (one pass over X),
