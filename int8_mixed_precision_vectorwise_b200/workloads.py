@@ -52,6 +52,12 @@ def bias(seed: int, N: int, std: float = 0.01) -> np.ndarray:
     return (g.standard_normal(N, dtype=np.float32) * np.float32(std)).astype(np.float16)
 
 
+def grad_output(seed: int, M: int, N: int) -> np.ndarray:
+    """dY fp16 [M, N] ~ N(0, 1): the gradient arriving at a layer's output."""
+    g = rng(seed)
+    return g.standard_normal((M, N), dtype=np.float32).astype(np.float16)
+
+
 @dataclass
 class Linear:
     """One Linear8bitLt call: X [M, K] -> out [M, N]."""

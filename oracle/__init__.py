@@ -11,4 +11,5 @@ from .llm_int8 import (  # noqa: F401
     int8_mm_dequant,
     dequant,
     linear8bit_forward,
+    linear8bit_backward_input,
 )

@@ -36,6 +36,11 @@ listed with its reason in the design notes of the repository):
                    + (SCB[n]/127) * sum_{j in O} x[i,j]*CB[n,j] )``
       evaluated in float64 with one final round to fp16; the outlier weights
       are the int8 weights dequantised (the boundary takes no fp16 weight).
+* R7  input gradient (training through the frozen int8 layer):
+      ``dX = fp16(dY . W^)`` evaluated in float64 with one final round, where
+      ``W^ = dequant(CB, SCB)`` is the fp16 dequantised weight.  This is the
+      chain rule for ``y = X . W^T + bias``; the pages only say that int8
+      modules carry trainable adapters, so the layer must pass gradients on.
 
 Precision: the quantisation decisions (R1-R4) are taken in IEEE fp32, the
 precision the GPU takes them in; everything after the integer product is
@@ -219,3 +224,24 @@ def linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, rows=None)
     Returns fp16 [M or len(rows), N].
     """
     return _forward_f64(X, CB, SCB, bias, threshold, rows).astype(np.float16)
+
+
+def linear8bit_backward_input(dY, CB, SCB, rows=None):
+    """Input gradient of the int8 linear layer (reading R7).
+
+    "`bitsandbytes` - `Linear8bitLt` integration into `transformers` models",
+    discussion of fine-tuning: trainable adapters sit on top of frozen int8
+    modules, so the gradient reaches the layer input through the dequantised
+    weight ``W^ = dequant(CB, SCB)``; the int8 weight gets no gradient.
+
+    Args:
+      dY: fp16 [M, N] gradient of the layer output; CB: int8 [N, K]; SCB: fp32 [N].
+      rows: optional row subset of dY to evaluate.
+
+    Returns fp16 [M or len(rows), K] = fp16(dY . W^) (float64 product, one rounding).
+    """
+    dY = _as_f16(dY)
+    if rows is not None:
+        dY = dY[np.asarray(rows, dtype=np.int64)]
+    W = dequant(CB, SCB).astype(np.float64)
+    return (dY.astype(np.float64) @ W).astype(np.float16)

@@ -313,3 +313,66 @@ def test_weight_quant_is_threshold_zero():
     CB, SCB = oracle.quantize_weight_rowwise(W)
     assert CB.tolist() == [[8, -4, 127], [0, 0, 0]]   # r = 127/8 = 15.875: 7.9375 -> 8, -3.96875 -> -4
     assert SCB.tolist() == [8.0, 0.0]
+
+
+# ---------------------------------------------------------------- input gradient
+def _frozen_layer(seed, M, N, K):
+    rng = np.random.default_rng(seed)
+    W = f16(rng.normal(0.0, 0.02, (N, K)))
+    CB, SCB = oracle.quantize_weight_rowwise(W)
+    dY = f16(rng.normal(0.0, 1.0, (M, N)))
+    return CB, SCB, dY
+
+
+@pytest.mark.parametrize("seed,M,N,K", [(0, 5, 24, 40), (1, 33, 64, 16), (2, 8, 17, 48)])
+def test_backward_input_is_autograd_gradient(seed, M, N, K):
+    """The oracle's dX equals what torch autograd derives for y = X . W^T + b in float64
+    (a transposed or mis-indexed product fails on these non-square shapes)."""
+    import torch
+    CB, SCB, dY = _frozen_layer(seed, M, N, K)
+    W = torch.from_numpy(oracle.dequant(CB, SCB).astype(np.float64))
+    X = torch.zeros((M, K), dtype=torch.float64, requires_grad=True)
+    b = torch.ones(N, dtype=torch.float64)
+    y = X @ W.T + b
+    (y * torch.from_numpy(dY.astype(np.float64))).sum().backward()
+    got = oracle.linear8bit_backward_input(dY, CB, SCB)
+    assert got.shape == (M, K)
+    assert np.array_equal(got, X.grad.numpy().astype(np.float16))
+
+
+def test_backward_input_one_hot_rows_select_weight_rows():
+    """dY = e_n picks row n of the dequantised weight, exactly."""
+    CB, SCB, _ = _frozen_layer(3, 1, 12, 32)
+    dY = f16(np.eye(12))
+    assert np.array_equal(oracle.linear8bit_backward_input(dY, CB, SCB), oracle.dequant(CB, SCB))
+
+
+def test_backward_input_brute_force():
+    """Exact rational sums with Python integers / fractions on a tiny case."""
+    CB, SCB, dY = _frozen_layer(4, 3, 5, 4)
+    W = oracle.dequant(CB, SCB)
+    got = oracle.linear8bit_backward_input(dY, CB, SCB)
+    for i in range(3):
+        for k in range(4):
+            s = sum(Fraction(float(dY[i, n])) * Fraction(float(W[n, k])) for n in range(5))
+            assert got[i, k] == np.float16(float(s))
+
+
+def test_backward_input_row_subset():
+    CB, SCB, dY = _frozen_layer(5, 9, 16, 32)
+    full = oracle.linear8bit_backward_input(dY, CB, SCB)
+    assert np.array_equal(oracle.linear8bit_backward_input(dY, CB, SCB, rows=[8, 0, 3]), full[[8, 0, 3]])
+
+
+def test_dequant_two_step_fp32_equals_one_rounding():
+    """For every code c in [-127, 127] and every positive finite fp16 row scale, evaluating
+    fp16(fl32(c * fl32(SCB / 127))) gives the oracle's once-rounded fp16(c * SCB / 127):
+    the exact value c * SCB / 127 never lies within 2^-18 (relative) of an fp16 rounding
+    boundary unless it is on one, and then it is representable.  So a GPU dequantiser that
+    takes those two fp32 steps can be compared with the oracle bit for bit."""
+    scb = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    s = scb / np.float32(127.0)
+    for c in range(-127, 128):
+        two = (np.float32(c) * s).astype(np.float16)
+        one = oracle.dequant(np.full((scb.size, 1), c, np.int8), scb)[:, 0]
+        assert np.array_equal(two.view(np.uint16), one.view(np.uint16)), c
