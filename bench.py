@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows per linear in the CPU oracle sample")
     return ap.parse_args()
 
@@ -224,6 +225,55 @@ def measure_decode(i8, torch, dev, st, world, dist, reps: int = 20):
             "peak_source": "of measured hbm_gbs" if measured_peaks() else "of fallback",
             "bytes": "N*K + 4N + 2MK + 2MN per call", "points": points,
             "best_GB/s": best["GB/s"], "best_frac": best["frac"]}
+
+
+def measure_backward(i8, torch, dev, st, world, dist, reps: int = 20):
+    """Input gradient through the frozen int8 layer for the distinct weight shapes of the
+    Llama-7B-shaped layer at 4096 tokens: the transposed dequantisation of the weight
+    (HBM-bound, 3NK bytes) and dX = dY . W^ on the fp16 tensor cores (2MNK flops), each
+    timed alone with CUDA events over `reps` back-to-back calls."""
+    layers = wl.workloads()["C3"].layers
+    peaks = measured_peaks()
+    f16_peak = float(peaks["bf16_tflops"]) if peaks else 1590.0
+    hbm = float(peaks["hbm_gbs"]) if peaks else 6650.0
+    points, seen = [], set()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(reps):
+            fn()
+        e1.record(st)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps * 1e3  # us per call
+
+    for li, L in enumerate(layers):
+        if (L.N, L.K) in seen:
+            continue
+        seen.add((L.N, L.K))
+        CB, SCB, _ = i8.i8_quantize_rowwise(torch.from_numpy(wl.weight(500 + li, L.N, L.K)).to(dev), 0.0)
+        dY = torch.from_numpy(wl.grad_output(600 + li, L.M, L.N)).to(dev)
+        Wt = torch.empty((L.K, L.N), dtype=torch.float16, device=dev)
+        dX = torch.empty((L.M, L.K), dtype=torch.float16, device=dev)
+        us_dq = timed(lambda: i8.i8_dequant_transposed(CB, SCB, Wt))
+        us_mm = timed(lambda: i8.i8_linear8bit_backward_input(dY, Wt, dX))
+        gbs = 3.0 * L.N * L.K / us_dq / 1e3
+        tflops = 2.0 * L.M * L.N * L.K / us_mm / 1e6
+        points.append({"layer": L.name, "dY": f"{L.M}x{L.N}", "W": f"{L.N}x{L.K}",
+                       "dequant_t_us": round(us_dq, 2), "dequant_t_GB/s": round(gbs, 1),
+                       "dequant_t_frac": round(gbs / hbm, 4),
+                       "gemm_us": round(us_mm, 2), "gemm_TFLOP/s": round(tflops, 1),
+                       "gemm_frac": round(tflops / f16_peak, 4)})
+    return {"metric": "input-gradient fp16 GEMM TFLOP/s (2MNK/s) and transposed dequant GB/s",
+            "gemm_peak_tflops": f16_peak, "hbm_peak_gbs": hbm,
+            "peak_source": ("of measured: fp16 = bf16_tflops (nominal fp16:bf16 = 1:1), hbm_gbs" if peaks
+                            else "of fallback: 1.59 PFLOP/s, 6.65 TB/s"),
+            "points": points}
 
 
 def cpu_threads() -> int:
@@ -443,6 +493,11 @@ def run_ours(args):
     if not args.no_decode:
         decode = measure_decode(i8, torch, dev, st, world, dist)
 
+    # ---- input gradient (training through the frozen int8 layer)
+    backward = None
+    if not args.no_backward:
+        backward = measure_backward(i8, torch, dev, st, world, dist)
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -503,6 +558,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "decode": decode,
+        "backward": backward,
         "clocks": clocks,
         "gpu_launches": K * n_launch_per_step,
         "gpu_launches_note": f"per step per linear: quantise + outlier prepare + GEMM ({gemm_launches} GEMMs)",

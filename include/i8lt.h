@@ -127,6 +127,34 @@ I8_API i8_status i8_dequant(const int8_t* CB, const float* SCB, int N, int K, i8
                      i8_stream_t stream);
 
 /*
+ * i8_dequant_transposed — the same dequantised weight stored transposed:
+ *   Wt[k, n] = fp16(CB[n, k] * SCB[n] / 127), bit for bit the transpose of
+ *   i8_dequant's W.  CB [N, K] int8, SCB [N] fp32, Wt [K, N] fp16 output.
+ * Requires K % 16 == 0 and N % 8 == 0 (16-byte rows of Wt); K <= 4194240.
+ * Wt is the weight operand of i8_linear8bit_backward_input.
+ */
+I8_API i8_status i8_dequant_transposed(const int8_t* CB, const float* SCB, int N, int K,
+                                i8_half* Wt, i8_stream_t stream);
+
+/*
+ * i8_linear8bit_backward_input — input gradient of the int8 linear layer:
+ *   dX[i, k] = fp16( sum_n dY[i, n] * Wt[k, n] ),  fp32 accumulation,
+ * i.e. dX = dY . W^ for y = X . W^T + bias with W^ = Wt^T.  With Wt from
+ * i8_dequant_transposed, W^ is the dequantised int8 weight, so the gradient
+ * flows through the frozen quantised layer to the layers and adapters before
+ * it ("`bitsandbytes` - `Linear8bitLt` integration into `transformers`
+ * models", discussion of fine-tuning with trainable adapters on top of int8
+ * modules; the int8 weight itself is not trained, so there is no weight
+ * gradient).  The product has no int8 part and no outlier decomposition: it
+ * runs on the tensor cores in fp16 (tcgen05 kind::f16).
+ *   dY [M, N] fp16, Wt [K, N] fp16, dX [M, K] fp16 output.
+ * Requires N % 8 == 0 (16-byte rows of dY and Wt).  A pipeline wait that ran
+ * past its time limit leaves dX unspecified and is not reported.
+ */
+I8_API i8_status i8_linear8bit_backward_input(const i8_half* dY, const i8_half* Wt, int M, int N,
+                                       int K, i8_half* dX, i8_stream_t stream);
+
+/*
  * Workspace bytes i8_linear8bit_forward needs for these sizes.  The workspace
  * is caller-owned device memory, 256-byte aligned, that holds CA, SCA, the
  * outlier bitmap / index list, the gathered fp16 outlier operands and the

@@ -10,8 +10,10 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     STATUS,
     i8_dequant,
+    i8_dequant_transposed,
     i8_int8_linear_matmul,
     i8_int8_mm_dequant,
+    i8_linear8bit_backward_input,
     i8_linear8bit_forward,
     i8_linear8bit_forward_static,
     i8_linear8bit_matmul_dequant,

@@ -32,7 +32,7 @@ EXPORTS = (
     "i8_status_string", "i8_quantize_rowwise", "i8_outlier_columns", "i8_int8_linear_matmul",
     "i8_int8_mm_dequant", "i8_dequant", "i8_linear8bit_workspace_size", "i8_linear8bit_forward",
     "i8_read_status", "i8_selftest_bounded_wait", "i8_linear8bit_prepare", "i8_linear8bit_matmul_dequant",
-    "i8_linear8bit_forward_static",
+    "i8_linear8bit_forward_static", "i8_dequant_transposed", "i8_linear8bit_backward_input",
 )
 
 
@@ -59,6 +59,8 @@ def _declare(lib):
         "i8_int8_linear_matmul": (_I, [_P, _P, _I, _I, _I, _P, _P]),
         "i8_int8_mm_dequant": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
         "i8_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
+        "i8_dequant_transposed": (_I, [_P, _P, _I, _I, _P, _P]),
+        "i8_linear8bit_backward_input": (_I, [_P, _P, _I, _I, _I, _P, _P]),
         "i8_linear8bit_workspace_size": (_S, [_I, _I, _I, _I]),
         "i8_linear8bit_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
         "i8_linear8bit_prepare": (_I, [_P, _P, _I, _I, _I, _F, _P, _S, _I, _P]),
@@ -176,6 +178,31 @@ def i8_dequant(CB, SCB, W=None):
     W = torch.empty((N, K), dtype=torch.float16, device=CB.device) if W is None else W
     _check("i8_dequant", lib().i8_dequant(_ptr(CB), _ptr(SCB), N, K, _ptr(W), _stream(CB.device)))
     return W
+
+
+def i8_dequant_transposed(CB, SCB, Wt=None):
+    """Wt = W^T with W = fp16(CB * SCB[n] / 127): CB [N, K] -> Wt [K, N]."""
+    _need(CB, torch.int8, "CB", 2)
+    _need(SCB, torch.float32, "SCB", 1)
+    N, K = CB.shape
+    Wt = torch.empty((K, N), dtype=torch.float16, device=CB.device) if Wt is None else Wt
+    _check("i8_dequant_transposed", lib().i8_dequant_transposed(
+        _ptr(CB), _ptr(SCB), N, K, _ptr(Wt), _stream(CB.device)))
+    return Wt
+
+
+def i8_linear8bit_backward_input(dY, Wt, dX=None):
+    """dX = fp16(dY . Wt^T): dY [M, N], Wt [K, N] (from i8_dequant_transposed) -> dX [M, K]."""
+    _need(dY, torch.float16, "dY", 2)
+    _need(Wt, torch.float16, "Wt", 2)
+    M, N = dY.shape
+    K = Wt.shape[0]
+    if Wt.shape[1] != N:
+        raise ValueError("dY and Wt must share N")
+    dX = torch.empty((M, K), dtype=torch.float16, device=dY.device) if dX is None else dX
+    _check("i8_linear8bit_backward_input", lib().i8_linear8bit_backward_input(
+        _ptr(dY), _ptr(Wt), M, N, K, _ptr(dX), _stream(dY.device)))
+    return dX
 
 
 def i8_linear8bit_workspace_size(M: int, N: int, K: int, max_outlier_cols: int) -> int:

@@ -33,6 +33,12 @@
 // with more, tcgen05 kind::f16 MMAs write D into TMEM columns [256,512) and
 // the accumulator is single-buffered.
 // The epilogue writes fp16 32x32 boxes through shared memory with TMA stores.
+//
+// A third mode runs the same pipeline as a plain fp16 GEMM, out = fp16(XO . WO^T)
+// with fp32 accumulation: every k-block is a kind::f16 block, the accumulator
+// is double-buffered in TMEM and the epilogue only rounds.  It computes the
+// input gradient dX = dY . W^ of a linear layer whose frozen weight W^ is the
+// dequantised int8 weight, with XO = dY [M, N] and WO = W^ transposed [K, N].
 #include <cuda_fp16.h>
 
 #include "kernels.cuh"
@@ -106,9 +112,11 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 
 }  // namespace
 
-template <bool RAW>
+template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_gemm_i8_tcgen05(const __grid_constant__ GemmMaps tm, const GemmArgs p) {
+  constexpr bool RAW = MODE == kGemmRaw;
+  constexpr bool F16 = MODE == kGemmF16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);  // used in the leader only
@@ -129,7 +137,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int num_m = (M + 2 * BM - 1) / (2 * BM);
   const int num_n = (N + BN - 1) / BN;
   const int tiles = num_m * num_n;
-  const int kb_int = (K + BK - 1) / BK;
+  const int kb_int = F16 ? 0 : (K + BK - 1) / BK;
   const Units U(tiles, npairs);
 
   if (threadIdx.x == 0) {
@@ -146,8 +154,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm.A);
-    tma_prefetch_desc(&tm.B);
+    if constexpr (F16) {
+      tma_prefetch_desc(&tm.XO);
+      tma_prefetch_desc(&tm.WO);
+    } else {
+      tma_prefetch_desc(&tm.A);
+      tma_prefetch_desc(&tm.B);
+    }
     if (!RAW && p.tma_store) tma_prefetch_desc(&tm.Out);
   }
   if (warp == 1) {
@@ -164,14 +177,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   // quantiser wrote, so wait for them here (a no-op without that overlap).
   pdl_wait();
   int n_used = 0;
-  if (!RAW && p.n_used != nullptr) n_used = min(max(*p.n_used, 0), p.out_cap);
+  if (!RAW && !F16 && p.n_used != nullptr) n_used = min(max(*p.n_used, 0), p.out_cap);
   // Up to 16 outlier columns are added by the epilogue with warp MMAs so the
   // TMEM accumulators stay double-buffered; more go through tcgen05 fp16 MMAs
-  // into a second accumulator.
-  const bool small_o = n_used > 0 && n_used <= SMALL_O && p.XO != nullptr && p.WO != nullptr;
-  const int kb_out = small_o ? 0 : (n_used + 63) / 64;
+  // into a second accumulator.  The fp16 mode has only fp16 k-blocks (K fp16
+  // columns) and double-buffers their accumulator.
+  const bool small_o = !F16 && n_used > 0 && n_used <= SMALL_O && p.XO != nullptr && p.WO != nullptr;
+  const int kb_out = F16 ? (K + 63) / 64 : (small_o ? 0 : (n_used + 63) / 64);
   const int kb_all = kb_int + kb_out;
-  const bool dbl = kb_out == 0;
+  const bool dbl = F16 || kb_out == 0;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -247,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (!mbar_wait_bounded(&acc_empty[buf], (use & 1u) ^ 1u, s_abort, p.status, p.wait_limit_ns)) break;
         tc_fence_after_sync();
         const uint32_t d_int = tmem_base + static_cast<uint32_t>(buf * BN);
-        const uint32_t d_fp = tmem_base + static_cast<uint32_t>(BN);
+        const uint32_t d_fp = tmem_base + static_cast<uint32_t>(F16 ? buf * BN : BN);
         bool ok = true;
         for (int kb = 0; kb < kb_all; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, s_abort, p.status, p.wait_limit_ns)) {
@@ -317,7 +331,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = row_base + g + 8 * i;
-        sa4[i] = (!RAW && r < M) ? __ldg(p.SCA + r) * (1.0f / 16129.0f) : 0.f;
+        sa4[i] = (!RAW && !F16 && r < M) ? __ldg(p.SCA + r) * (1.0f / 16129.0f) : 0.f;
       }
       // Few outliers: the A fragments (X[:, O] rows) of the 16-wide outlier
       // product.  The gathered operands store each group of 16 outlier columns
@@ -349,7 +363,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t bf_n[4][2];
       auto fetch_chunk = [&](int cc) {
         const int n = n0 + cc * 32 + lane;
-        const bool in = !RAW && n < N;
+        const bool in = !RAW && !F16 && n < N;
         sb_n = in ? __ldg(p.SCB + n) : 0.f;
         bi_n = (in && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
 #pragma unroll
@@ -383,12 +397,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         if (cc + 1 < nch) fetch_chunk(cc + 1);
         uint32_t c[2][16];  // int32 accumulators of row blocks 0 / 1
-        tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
-        tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
-        uint32_t f[2][16];  // fp32 outlier accumulators (many-outlier path)
-        if (!RAW && kb_out > 0) {
-          tmem_ld_16x256b_x4(t_fp + cc * 32, f[0]);
-          tmem_ld_16x256b_x4(t_fp + (16u << 16) + cc * 32, f[1]);
+        if constexpr (!F16) {
+          tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
+          tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
+        }
+        // fp32 accumulators: the outlier product (many-outlier path) or, in the
+        // fp16 mode, the whole product (in the double-buffered columns)
+        uint32_t f[2][16];
+        if (F16 || (!RAW && kb_out > 0)) {
+          const uint32_t t_f = F16 ? t_int : t_fp;
+          tmem_ld_16x256b_x4(t_f + cc * 32, f[0]);
+          tmem_ld_16x256b_x4(t_f + (16u << 16) + cc * 32, f[1]);
         }
         tmem_wait_ld();
         const int nb = n0 + cc * 32;
@@ -417,10 +436,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           const int j = cb * 8 + 2 * tq;
-          const float sb0 = __shfl_sync(0xffffffffu, sb_c, j);
-          const float sb1 = __shfl_sync(0xffffffffu, sb_c, j + 1);
-          const float b0 = __shfl_sync(0xffffffffu, bi_c, j);
-          const float b1 = __shfl_sync(0xffffffffu, bi_c, j + 1);
+          float sb0 = 0.f, sb1 = 0.f, b0 = 0.f, b1 = 0.f;
+          if constexpr (!F16) {
+            sb0 = __shfl_sync(0xffffffffu, sb_c, j);
+            sb1 = __shfl_sync(0xffffffffu, sb_c, j + 1);
+            b0 = __shfl_sync(0xffffffffu, bi_c, j);
+            b1 = __shfl_sync(0xffffffffu, bi_c, j + 1);
+          }
 #pragma unroll
           for (int rb = 0; rb < 2; ++rb) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -432,12 +454,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-              const float sa = sa4[2 * rb + hh];
-              const float v0 = fmaf(d[2 * hh], sb0 * (1.0f / 127.0f),
-                                    fmaf(static_cast<float>(static_cast<int32_t>(c[rb][4 * cb + 2 * hh])), sa * sb0, b0));
-              const float v1 = fmaf(d[2 * hh + 1], sb1 * (1.0f / 127.0f),
-                                    fmaf(static_cast<float>(static_cast<int32_t>(c[rb][4 * cb + 2 * hh + 1])), sa * sb1, b1));
-              halves[rb][cb][hh] = pack_half2(v0, v1);
+              if constexpr (F16) {
+                halves[rb][cb][hh] = pack_half2(d[2 * hh], d[2 * hh + 1]);
+              } else {
+                const float sa = sa4[2 * rb + hh];
+                const float v0 = fmaf(d[2 * hh], sb0 * (1.0f / 127.0f),
+                                      fmaf(static_cast<float>(static_cast<int32_t>(c[rb][4 * cb + 2 * hh])), sa * sb0, b0));
+                const float v1 = fmaf(d[2 * hh + 1], sb1 * (1.0f / 127.0f),
+                                      fmaf(static_cast<float>(static_cast<int32_t>(c[rb][4 * cb + 2 * hh + 1])), sa * sb1, b1));
+                halves[rb][cb][hh] = pack_half2(v0, v1);
+              }
             }
           }
         }
@@ -502,13 +528,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 }
 
-// Number of CTA pairs that fit on the device at once (cached per device).
-static int max_pairs(bool raw, int num_sms) {
-  static int cache[2][64] = {{0}};
+using GemmKernel = void (*)(GemmMaps, GemmArgs);
+
+static GemmKernel gemm_kernel(GemmMode mode) {
+  switch (mode) {
+    case kGemmRaw: return k_gemm_i8_tcgen05<kGemmRaw>;
+    case kGemmF16: return k_gemm_i8_tcgen05<kGemmF16>;
+    default: return k_gemm_i8_tcgen05<kGemmFused>;
+  }
+}
+
+// Number of CTA pairs that fit on the device at once (cached per mode and device).
+static int max_pairs(GemmMode mode, int num_sms) {
+  static int cache[3][64] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
-  const int r = raw ? 1 : 0;
-  if (dev >= 0 && dev < 64 && cache[r][dev] > 0) return cache[r][dev];
+  const int m = static_cast<int>(mode);
+  if (dev >= 0 && dev < 64 && cache[m][dev] > 0) return cache[m][dev];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1), 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
@@ -521,29 +557,26 @@ static int max_pairs(bool raw, int num_sms) {
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int n = 0;
-  cudaError_t e = raw ? cudaOccupancyMaxActiveClusters(&n, k_gemm_i8_tcgen05<true>, &cfg)
-                      : cudaOccupancyMaxActiveClusters(&n, k_gemm_i8_tcgen05<false>, &cfg);
+  cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel(mode), &cfg);
   if (e != cudaSuccess || n <= 0) {
     cudaGetLastError();
     n = num_sms / 2;
   }
-  if (dev >= 0 && dev < 64) cache[r][dev] = n;
+  if (dev >= 0 && dev < 64) cache[m][dev] = n;
   return n;
 }
 
-cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, bool raw_int32, int num_sms, cudaStream_t st) {
-  static bool attr_done[2] = {false, false};
-  const int raw = raw_int32 ? 1 : 0;
-  if (!attr_done[raw]) {
-    cudaError_t e = raw ? cudaFuncSetAttribute(k_gemm_i8_tcgen05<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               SMEM_ALLOC)
-                        : cudaFuncSetAttribute(k_gemm_i8_tcgen05<false>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, GemmMode mode, int num_sms, cudaStream_t st) {
+  if (mode != kGemmFused && mode != kGemmRaw && mode != kGemmF16) return cudaErrorInvalidValue;
+  static bool attr_done[3] = {false, false, false};
+  const int m = static_cast<int>(mode);
+  if (!attr_done[m]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel(mode), cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    attr_done[raw] = true;
+    attr_done[m] = true;
   }
   const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
-  const int pairs_fit = max_pairs(raw_int32, num_sms);
+  const int pairs_fit = max_pairs(mode, num_sms);
   // fewer tiles than pairs: run each tile as two half tiles where that fits
   const int pairs = tiles >= pairs_fit ? pairs_fit : (2 * tiles <= pairs_fit ? 2 * tiles : tiles);
   cudaLaunchConfig_t cfg = {};
@@ -556,8 +589,7 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, bool raw_int32,
   attr.val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  return raw_int32 ? cudaLaunchKernelEx(&cfg, k_gemm_i8_tcgen05<true>, maps, a)
-                   : cudaLaunchKernelEx(&cfg, k_gemm_i8_tcgen05<false>, maps, a);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel(mode), maps, a);
 }
 
 // ------------------------------------------------------------------ self test

@@ -145,7 +145,33 @@ i8_status run_gemm(const int8_t* A, const int8_t* B, int M, int N, int K, GemmAr
   }
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
-  return cuda_status(i8lt::launch_gemm(maps, args, raw, sms, st));
+  return cuda_status(i8lt::launch_gemm(maps, args, raw ? i8lt::kGemmRaw : i8lt::kGemmFused, sms, st));
+}
+
+// out [M, Nout] = fp16(Aop [M, Kc] . Bop [Nout, Kc]^T), fp16 operands, fp32 accumulation.
+i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, int Kc, __half* out, cudaStream_t st) {
+  i8lt::GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const uint64_t ld_bytes = static_cast<uint64_t>(Kc) * 2;
+  if (!encode_2d(&maps.XO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Aop, Kc, M, ld_bytes, 64, i8lt::kGemmBM) ||
+      !encode_2d(&maps.WO, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Bop, Kc, Nout, ld_bytes, 64, i8lt::kGemmBN / 2))
+    return I8_ERR_CUDA;
+  GemmArgs a{};
+  a.M = M;
+  a.N = Nout;
+  a.K = Kc;
+  a.out = out;
+  a.wait_limit_ns = kWaitLimitNs;
+  a.tma_store = 0;
+  if (Nout % 8 == 0) {
+    if (!encode_2d(&maps.Out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, out, Nout, M, static_cast<uint64_t>(Nout) * 2,
+                   i8lt::kGemmOutBox, i8lt::kGemmOutBox, CU_TENSOR_MAP_SWIZZLE_64B))
+      return I8_ERR_CUDA;
+    a.tma_store = 1;
+  }
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_gemm(maps, a, i8lt::kGemmF16, sms, st));
 }
 
 }  // namespace
@@ -383,6 +409,26 @@ i8_status i8_dequant(const int8_t* CB, const float* SCB, int N, int K, i8_half* 
   if (sms <= 0) return I8_ERR_CUDA;
   return cuda_status(i8lt::launch_dequant(CB, SCB, N, K, reinterpret_cast<__half*>(W), sms,
                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_dequant_transposed(const int8_t* CB, const float* SCB, int N, int K, i8_half* Wt,
+                                i8_stream_t stream) {
+  if (!CB || !SCB || !Wt) return I8_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % 8 != 0 || K > 65535 * 64) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(CB) || !aligned16(Wt)) return I8_ERR_UNSUPPORTED_SHAPE;
+  return cuda_status(i8lt::launch_dequant_t(CB, SCB, N, K, reinterpret_cast<__half*>(Wt),
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_linear8bit_backward_input(const i8_half* dY, const i8_half* Wt, int M, int N, int K, i8_half* dX,
+                                       i8_stream_t stream) {
+  if (!dY || !Wt || !dX) return I8_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (N % 8 != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(dY) || !aligned16(Wt) || !aligned16(dX)) return I8_ERR_UNSUPPORTED_SHAPE;
+  return run_gemm_f16(reinterpret_cast<const __half*>(dY), reinterpret_cast<const __half*>(Wt), M, K, N,
+                      reinterpret_cast<__half*>(dX), reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_cols) {

@@ -22,6 +22,8 @@ cudaError_t launch_mm_dequant(const int32_t* C, const float* SCA, const float* S
                               int N, __half* out, int num_sms, cudaStream_t st);
 cudaError_t launch_dequant(const int8_t* CB, const float* SCB, int N, int K, __half* W, int num_sms,
                            cudaStream_t st);
+// Wt [K, N] = the transpose of launch_dequant's W (K % 16 == 0, N % 8 == 0).
+cudaError_t launch_dequant_t(const int8_t* CB, const float* SCB, int N, int K, __half* Wt, cudaStream_t st);
 
 // Tensor-core GEMM (tcgen05, TMA-fed, TMEM accumulators).
 struct GemmArgs {
@@ -54,8 +56,15 @@ struct GemmMaps {
 
 constexpr int kSmallOutliers = 16;
 
+// What one launch of the GEMM computes:
+//   kGemmFused  out = fp16 LLM.int8() forward (int8 codes A/B, outlier operands XO/WO, scales, bias)
+//   kGemmRaw    C = A . B^T as int32
+//   kGemmF16    out = fp16(XO . WO^T), an fp16 GEMM with fp32 accumulation over K fp16
+//               columns: XO [M, K] and WO [N, K] (the A/B maps and every scale are unused)
+enum GemmMode : int { kGemmFused = 0, kGemmRaw = 1, kGemmF16 = 2 };
+
 // The kernel runs on CTA pairs.
-cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, bool raw_int32, int num_sms, cudaStream_t st);
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, GemmMode mode, int num_sms, cudaStream_t st);
 
 // Box sizes the tensor maps above must be encoded with.
 constexpr int kGemmBM = 128;        // rows of A per CTA (a CTA pair covers 256 rows)

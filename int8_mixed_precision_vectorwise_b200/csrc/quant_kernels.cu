@@ -7,6 +7,7 @@
 //                       columns, gather X[:, O] and fp16(CB[:, O]) for the outlier product
 //   k_mm_dequant        int32 -> fp16 with row x column scales / 127^2 + bias
 //   k_dequant           int8 weight -> fp16 ("Next steps": int8 dequantize op)
+//   k_dequant_t         the same, stored transposed (operand of the input-gradient GEMM)
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -396,6 +397,43 @@ __global__ void __launch_bounds__(256) k_dequant(const int8_t* __restrict__ CB, 
   }
 }
 
+// The same dequantised weight, stored transposed: Wt[k, n] = fp16(CB[n, k] * SCB[n] / 127)
+// (the operand the input-gradient GEMM reads K-major).  One 64 x 64 tile per
+// block through shared memory: each thread reads 16 codes of one weight row and
+// writes them as a column of the tile; the tile leaves as 16-byte rows of Wt.
+// Requires K % 16 == 0 (a 16-code vector is all inside or all outside) and
+// N % 8 == 0 (likewise for an 8-value vector of a Wt row).
+constexpr int kDqT = 64;
+
+__global__ void __launch_bounds__(256) k_dequant_t(const int8_t* __restrict__ CB, const float* __restrict__ SCB,
+                                                   int N, int K, __half* __restrict__ Wt) {
+  __shared__ __align__(16) __half t[kDqT][kDqT + 8];  // [k][n]; 144-byte rows keep 16-byte alignment
+  const int n0 = blockIdx.x * kDqT, k0 = blockIdx.y * kDqT;
+  {
+    // lanes of a warp take consecutive weight rows, so their column writes to
+    // the tile fall in distinct banks
+    const int r = threadIdx.x & (kDqT - 1), c = (threadIdx.x >> 6) * 16;
+    const int n = n0 + r, k = k0 + c;
+    int4 v = make_int4(0, 0, 0, 0);
+    float sc = 0.f;
+    if (n < N && k < K) {
+      v = __ldcs(reinterpret_cast<const int4*>(CB + static_cast<size_t>(n) * K + k));
+      sc = __fdiv_rn(__ldg(SCB + n), 127.0f);
+    }
+    const int8_t* b = reinterpret_cast<const int8_t*>(&v);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) t[c + e][r] = __float2half_rn(static_cast<float>(b[e]) * sc);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = threadIdx.x; q < kDqT * (kDqT / 8); q += 256) {
+    const int kr = q >> 3, nc = (q & 7) * 8;
+    const int k = k0 + kr, n = n0 + nc;
+    if (k < K && n < N)
+      *reinterpret_cast<uint4*>(Wt + static_cast<size_t>(k) * N + n) = *reinterpret_cast<const uint4*>(&t[kr][nc]);
+  }
+}
+
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
                               cudaStream_t st) {
@@ -461,6 +499,13 @@ cudaError_t launch_dequant(const int8_t* CB, const float* SCB, int N, int K, __h
   const size_t nq = static_cast<size_t>(N) * K / 16;
   const int blocks = static_cast<int>(std::min<size_t>((nq + 255) / 256, static_cast<size_t>(num_sms) * 16));
   k_dequant<<<max(blocks, 1), 256, 0, st>>>(CB, SCB, N, K, W);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_t(const int8_t* CB, const float* SCB, int N, int K, __half* Wt, cudaStream_t st) {
+  const dim3 grid((N + kDqT - 1) / kDqT, (K + kDqT - 1) / kDqT, 1);
+  if (grid.y > 65535u) return cudaErrorInvalidConfiguration;
+  k_dequant_t<<<grid, 256, 0, st>>>(CB, SCB, N, K, Wt);
   return cudaGetLastError();
 }
 

@@ -27,7 +27,8 @@ def lib():
 def test_header_declares_expected_entry_points():
     names = declared_functions()
     for must in ("i8_quantize_rowwise", "i8_linear8bit_forward", "i8_dequant", "i8_int8_linear_matmul",
-                 "i8_int8_mm_dequant", "i8_read_status"):
+                 "i8_int8_mm_dequant", "i8_read_status", "i8_dequant_transposed",
+                 "i8_linear8bit_backward_input"):
         assert must in names
 
 
@@ -100,4 +101,19 @@ def test_other_rejects(lib):
     assert lib.i8_outlier_columns(None, 16, FAKE, 4, FAKE, None) == 1
     assert lib.i8_outlier_columns(FAKE, 16, None, 4, FAKE, None) == 1
     assert lib.i8_selftest_bounded_wait(FAKE, 10, None) == 1
+
+
+def test_backward_rejects(lib):
+    f = lib.i8_dequant_transposed
+    assert f(None, FAKE, 8, 16, FAKE, None) == 1
+    assert f(FAKE, FAKE, 0, 16, FAKE, None) == 1
+    assert f(FAKE, FAKE, 8, 24, FAKE, None) == 2      # K % 16
+    assert f(FAKE, FAKE, 12, 16, FAKE, None) == 2     # N % 8
+    assert f(FAKE, FAKE, 8, 16, FAKE_MIS, None) == 2
+    g = lib.i8_linear8bit_backward_input
+    assert g(None, FAKE, 4, 8, 16, FAKE, None) == 1
+    assert g(FAKE, FAKE, 4, 8, 16, None, None) == 1
+    assert g(FAKE, FAKE, 4, 0, 16, FAKE, None) == 1
+    assert g(FAKE, FAKE, 4, 12, 16, FAKE, None) == 2  # N % 8
+    assert g(FAKE, FAKE_MIS, 4, 8, 16, FAKE, None) == 2
     assert lib.i8_read_status(None, None, None) == 1

@@ -330,3 +330,74 @@ def test_forward_cuda_graph_replay(i8, M, N, K, n_out):
         _, _, cols = oracle.quantize_rowwise(X, 6.0)
         assert i8.i8_read_status(ws) == (0, len(cols))
         assert_close(host(out), oracle.linear8bit_forward(X, rCB, rSCB, b, 6.0), "graph replay")
+
+
+# ------------------------------------------------------------------ input gradient
+@pytest.mark.parametrize("N,K", [(8, 16), (200, 48), (1000, 2064), (4096, 4096), (11008, 4096), (4096, 11008)])
+def test_dequant_transposed_bit_exact(i8, N, K):
+    """Wt = dequant(CB, SCB)^T bit for bit (the fp32 two-step evaluation equals the oracle's
+    single rounding for every code and scale, so no tolerance is needed)."""
+    W = wl.weight(N * 3 + K, N, K)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    dCB, dSCB = dev(rCB), dev(rSCB)
+    Wt = host(i8.i8_dequant_transposed(dCB, dSCB))
+    ref = np.ascontiguousarray(oracle.dequant(rCB, rSCB).T)
+    assert Wt.shape == (K, N)
+    assert np.array_equal(Wt.view(np.uint16), ref.view(np.uint16))
+    assert np.array_equal(Wt.T, host(i8.i8_dequant(dCB, dSCB)))
+
+
+def assert_grad_close(got, ref, dY, W_hat, what=""):
+    """|gpu - oracle| <= n * 2^-23 * sum_n |dY[i, n] W^[n, k]| + ulp16: fp32 accumulation of
+    exact fp16 x fp16 products in any order (a per-add error of at most 2^-23, allowing
+    truncating adds), then one fp16 rounding on each side."""
+    g = np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape
+    n = dY.shape[1]
+    S = np.abs(dY.astype(np.float64)) @ np.abs(W_hat.astype(np.float64))
+    ulp = np.spacing(np.maximum(np.abs(g), np.abs(r)).astype(np.float16)).astype(np.float64)
+    bound = n * 2.0 ** -23 * S + ulp
+    d = np.abs(g - r)
+    bad = d > bound
+    if bad.any():
+        i = tuple(np.argwhere(bad)[0])
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} out of bound; first {i} got {g[i]} "
+                             f"want {r[i]} bound {bound[i]:.3g}; max abs {d.max():.3g}")
+
+
+BSHAPES = [(1, 8, 16), (130, 72, 48), (512, 1024, 768), (1024, 4096, 4096), (2048, 4096, 4096),
+           (300, 4104, 528), (4096, 4096, 11008)]
+
+
+@pytest.mark.parametrize("M,N,K", BSHAPES)
+def test_backward_input(i8, M, N, K):
+    """dX = dY . dequant(CB, SCB) through the tcgen05 fp16 GEMM, against the oracle."""
+    dY = wl.grad_output(M + 2 * N + 3 * K, M, N)
+    W = wl.weight(M + N + K, N, K)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    Wt = i8.i8_dequant_transposed(dev(rCB), dev(rSCB))
+    dX = host(i8.i8_linear8bit_backward_input(dev(dY), Wt))
+    rows = None if M <= 2048 else np.random.default_rng(M).choice(M, 256, replace=False)
+    ref = oracle.linear8bit_backward_input(dY, rCB, rSCB, rows=rows)
+    sel = dY if rows is None else dY[rows]
+    assert_grad_close(dX if rows is None else dX[rows], ref, sel, oracle.dequant(rCB, rSCB), "backward_input")
+
+
+def test_backward_input_plain_store_edge(i8):
+    """An output width that is not a multiple of 8 takes the plain-store epilogue."""
+    M, N, K = 100, 64, 20
+    dY = wl.grad_output(7, M, N)
+    rCB, rSCB = oracle.quantize_weight_rowwise(wl.weight(8, N, K))
+    W_hat = oracle.dequant(rCB, rSCB)
+    dX = host(i8.i8_linear8bit_backward_input(dev(dY), dev(np.ascontiguousarray(W_hat.T))))
+    assert_grad_close(dX, oracle.linear8bit_backward_input(dY, rCB, rSCB), dY, W_hat, "plain store")
+
+
+def test_backward_input_repeat_is_deterministic(i8):
+    dY = dev(wl.grad_output(9, 640, 2048))
+    rCB, rSCB = oracle.quantize_weight_rowwise(wl.weight(10, 2048, 1536))
+    Wt = i8.i8_dequant_transposed(dev(rCB), dev(rSCB))
+    a = host(i8.i8_linear8bit_backward_input(dY, Wt))
+    b = host(i8.i8_linear8bit_backward_input(dY, Wt))
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
