@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-other", action="store_true", help="skip the single-linear, OPT MLP and outlier sweep")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows per linear in the CPU oracle sample")
     return ap.parse_args()
 
@@ -276,6 +277,103 @@ def measure_backward(i8, torch, dev, st, world, dist, reps: int = 20):
             "points": points}
 
 
+def measure_other(i8, torch, dev, st, world, dist, reps: int = 50):
+    """The other workload families, each forward timed alone with CUDA events over `reps`
+    back-to-back calls (3 warm-up calls first):
+      - the single 16x1024 -> 1024 linear, launch-latency bound: eager, and the same call
+        captured once in a CUDA graph and replayed;
+      - the OPT-350m-shaped MLP pair at 512 tokens (fc2 fed the ReLU of the GPU's fc1 output,
+        computed before timing);
+      - the Llama-13B MLP shape 2048x5120 -> 13824 over outlier fractions {0, 0.1, 1, 5} %
+        and thresholds {0, 6} (one weight for all points), which exercises the many-outlier
+        tcgen05 fp16 path above 16 columns."""
+    W = wl.workloads()
+    peaks = measured_peaks()
+    peak = 2.0 * float(peaks["bf16_tflops"]) if peaks else 3180.0
+
+    def run(L, dX, CB, SCB, db, out, ws):
+        i8.i8_linear8bit_forward(dX, CB, SCB, db, L.threshold, out=out, workspace=ws,
+                                 max_outlier_cols=MAX_OUTLIER_COLS)
+
+    def timed(fn, n=reps):
+        for _ in range(3):
+            fn()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(n):
+            fn()
+        e1.record(st)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n * 1e3
+
+    def prepared(key, li, L, X=None, weight=None):
+        Xh, _, Wh, b = wl.layer_inputs(wl.seed_of(key), li, L)
+        if weight is None:
+            CB, SCB, _ = i8.i8_quantize_rowwise(torch.from_numpy(Wh).to(dev), 0.0)
+        else:
+            CB, SCB = weight
+        dX = X if X is not None else torch.from_numpy(Xh).to(dev)
+        db = None if b is None else torch.from_numpy(b).to(dev)
+        out = torch.empty((L.M, L.N), dtype=torch.float16, device=dev)
+        ws = torch.empty((i8.i8_linear8bit_workspace_size(L.M, L.N, L.K, MAX_OUTLIER_COLS),),
+                         dtype=torch.uint8, device=dev)
+        return dX, CB, SCB, db, out, ws
+
+    def status(ws):
+        code, count = i8.i8_read_status(ws)
+        if code != 0:
+            raise RuntimeError(f"device status {i8.STATUS.get(code, code)}")
+        return count
+
+    res = {"peak_tops": peak, "peak_source": ("of measured: int8 = 2 x bf16_tflops" if peaks
+                                              else "of fallback: int8 = 2 x 1.59 PFLOP/s")}
+    # single linear: eager and graph-replayed
+    L = W["C1"].layers[0]
+    a = prepared("C1", 0, L)
+    us_eager = timed(lambda: run(L, *a))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run(L, *a)
+    us_graph = timed(graph.replay)
+    del graph
+    res["single_linear"] = {"shape": f"{L.M}x{L.K}->{L.N}", "outlier_cols": status(a[5]),
+                            "us_eager": round(us_eager, 2), "us_graph": round(us_graph, 2),
+                            "TOPS_eager": round(L.ops / us_eager / 1e6, 2)}
+    # OPT-350m MLP pair
+    fc1, fc2 = W["C2"].layers
+    a1 = prepared("C2", 0, fc1)
+    run(fc1, *a1)
+    x2 = torch.relu(a1[4]).contiguous()
+    a2 = prepared("C2", 1, fc2, X=x2)
+    us1 = timed(lambda: run(fc1, *a1))
+    us2 = timed(lambda: run(fc2, *a2))
+    res["opt350m_mlp"] = {"fc1": {"shape": f"{fc1.M}x{fc1.K}->{fc1.N}", "outlier_cols": status(a1[5]),
+                                  "us": round(us1, 2), "TOPS": round(fc1.ops / us1 / 1e6, 1)},
+                          "fc2": {"shape": f"{fc2.M}x{fc2.K}->{fc2.N}", "outlier_cols": status(a2[5]),
+                                  "us": round(us2, 2), "TOPS": round(fc2.ops / us2 / 1e6, 1)}}
+    # Llama-13B MLP outlier sweep
+    keys = [k for k in W if k.startswith("C5_")]
+    weight = None
+    points = []
+    for key in keys:
+        L = W[key].layers[0]
+        if weight is None:
+            _, _, Wh, _ = wl.layer_inputs(wl.seed_of(keys[0]), 0, L)
+            CB, SCB, _ = i8.i8_quantize_rowwise(torch.from_numpy(Wh).to(dev), 0.0)
+            weight = (CB, SCB)
+        a = prepared(key, 0, L, weight=weight)
+        us = timed(lambda: run(L, *a), n=20)
+        tops = L.ops / us / 1e6
+        points.append({"key": key, "threshold": L.threshold, "planted_cols": L.n_out,
+                       "outlier_cols": status(a[5]), "us": round(us, 2), "TOPS": round(tops, 1),
+                       "frac": round(tops / peak, 4)})
+    res["llama13b_mlp_sweep"] = {"shape": "2048x5120->13824", "points": points}
+    return res
+
+
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -498,6 +596,11 @@ def run_ours(args):
     if not args.no_backward:
         backward = measure_backward(i8, torch, dev, st, world, dist)
 
+    # ---- the other workload families (single linear, OPT MLP, outlier sweep)
+    other_wl = None
+    if not args.no_other:
+        other_wl = measure_other(i8, torch, dev, st, world, dist)
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -559,6 +662,7 @@ def run_ours(args):
         "e2e": e2e,
         "decode": decode,
         "backward": backward,
+        "other_workloads": other_wl,
         "clocks": clocks,
         "gpu_launches": K * n_launch_per_step,
         "gpu_launches_note": f"per step per linear: quantise + outlier prepare + GEMM ({gemm_launches} GEMMs)",
