@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-other", action="store_true", help="skip the single-linear, OPT MLP and outlier sweep")
+    ap.add_argument("--no-shared", action="store_true", help="skip the shared-input layer step")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows per linear in the CPU oracle sample")
     return ap.parse_args()
 
@@ -374,6 +375,61 @@ def measure_other(i8, torch, dev, st, world, dist, reps: int = 50):
     return res
 
 
+def measure_shared_inputs(i8, torch, dev, st, world, dist, layers, reps: int = 20):
+    """The headline's seven linears fed the way a decoder layer feeds them: q/k/v read one X
+    and gate/up read one X, so each of those groups is one i8_linear8bit_forward_multi call
+    (X quantised and its outlier columns found once); o and down stay single forwards.  Same
+    weights, shapes and ops as the headline step; the inputs of k, v and up are q's and
+    gate's."""
+    by = {d["L"].name: d for d in layers}
+    groups = [["q_proj", "k_proj", "v_proj"], ["o_proj"], ["gate_proj", "up_proj"], ["down_proj"]]
+    if any(n not in by for g in groups for n in g) or len(layers) != 7:
+        return None
+    plan, launches = [], 0
+    for names in groups:
+        ds = [by[n] for n in names]
+        L0 = ds[0]["L"]
+        ws = None
+        if len(ds) > 1:
+            ws = torch.empty((i8.i8_linear8bit_multi_workspace_size(L0.M, L0.K, [d["L"].N for d in ds],
+                                                                    MAX_OUTLIER_COLS),), dtype=torch.uint8, device=dev)
+        plan.append((ds, ws))
+        launches += 3 + 2 * (len(ds) - 1)   # quantise, prepare, GEMM; per further weight: gather + GEMM
+
+    def step():
+        for ds, ws in plan:
+            L0 = ds[0]["L"]
+            if ws is None:
+                d = ds[0]
+                i8.i8_linear8bit_forward(d["X"], d["CB"], d["SCB"], d["b"], L0.threshold, out=d["out"],
+                                         workspace=d["ws"], max_outlier_cols=MAX_OUTLIER_COLS)
+            else:
+                i8.i8_linear8bit_forward_multi(ds[0]["X"], [d["CB"] for d in ds], [d["SCB"] for d in ds],
+                                               [d["b"] for d in ds], L0.threshold, outs=[d["out"] for d in ds],
+                                               workspace=ws, max_outlier_cols=MAX_OUTLIER_COLS)
+
+    for _ in range(3):
+        step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(reps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    for ds, ws in plan:
+        code, _ = i8.i8_read_status(ws if ws is not None else ds[0]["ws"])
+        if code != 0:
+            raise RuntimeError(f"device status {i8.STATUS.get(code, code)}")
+    ms = e0.elapsed_time(e1) / reps
+    ops = sum(d["L"].ops for d in layers)
+    return {"metric": "TOPS (2MNK/s) of the same seven linears with q/k/v and gate/up sharing their input",
+            "ms_per_step": ms, "TOPS": ops / ms / 1e9, "steps": reps, "gpu_launches_per_step": launches,
+            "calls": "forward_multi(q,k,v) + forward(o) + forward_multi(gate,up) + forward(down)"}
+
+
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -519,6 +575,11 @@ def run_ours(args):
     gemm_ms = sum(a.elapsed_time(b) for row in ev for a, b in row)
     ms_max = max_over_ranks(ms, world, dist, dev)
 
+    # ---- the same step with the inputs shared as in a decoder layer (informational)
+    shared = None
+    if not args.no_shared and args.workload == "C3":
+        shared = measure_shared_inputs(i8, torch, dev, st, world, dist, layers)
+
     # ---- end to end: host inputs -> device -> forward -> host outputs, per step
     e2e = None
     if not args.no_e2e:
@@ -663,6 +724,7 @@ def run_ours(args):
         "decode": decode,
         "backward": backward,
         "other_workloads": other_wl,
+        "shared_inputs": shared,
         "clocks": clocks,
         "gpu_launches": K * n_launch_per_step,
         "gpu_launches_note": f"per step per linear: quantise + outlier prepare + GEMM ({gemm_launches} GEMMs)",

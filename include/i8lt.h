@@ -192,6 +192,34 @@ I8_API i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const
                                 int max_outlier_cols, i8_stream_t stream);
 
 /*
+ * Several linear layers that read the same input X, as the query/key/value
+ * projections (or the gate/up projections) of a transformer block do once
+ * every nn.Linear is a Linear8bitLt ("`bitsandbytes` - `Linear8bitLt`
+ * integration into `transformers` models", which replaces all of a model's
+ * linear layers):
+ *   out[g] = Linear8bitLt(X; CB[g], SCB[g], bias[g]),  g = 0 .. G-1,
+ * each bit for bit what i8_linear8bit_forward returns for that weight alone.
+ * The outlier columns are a property of X (any |x| at or above the threshold
+ * in the column), so X is quantised, its outlier set found and X[:, O]
+ * gathered once for all G weights; then each weight gets its outlier rows
+ * fp16(CB[g][:, O]) and its own GEMM launch, in order g = 0 .. G-1.
+ *   X [M, K] fp16 device pointer.  CB, SCB, bias, N, out are HOST arrays of
+ *   G entries holding device pointers (bias may be NULL, or hold NULL
+ *   entries); CB[g] [N[g], K] int8, SCB[g] [N[g]] fp32, out[g] [M, N[g]] fp16.
+ *   1 <= G <= 16.  Every weight must pass i8_linear8bit_forward's checks.
+ * The workspace comes from i8_linear8bit_multi_workspace_size; status and
+ * outlier count are read with i8_read_status, as for the single forward.
+ */
+I8_API size_t i8_linear8bit_multi_workspace_size(int M, int K, int G, const int* N,
+                                          int max_outlier_cols);
+I8_API i8_status i8_linear8bit_forward_multi(const i8_half* X, int M, int K, int G,
+                                      const int8_t* const* CB, const float* const* SCB,
+                                      const i8_half* const* bias, const int* N,
+                                      i8_half* const* out, float threshold, void* workspace,
+                                      size_t workspace_bytes, int max_outlier_cols,
+                                      i8_stream_t stream);
+
+/*
  * The two halves of i8_linear8bit_forward, for callers that want to place
  * work or events between them (same arguments, same workspace, same stream):
  *   i8_linear8bit_prepare: resets the status word, quantises X into the

@@ -15,8 +15,10 @@ from ._binding import (  # noqa: F401
     i8_int8_mm_dequant,
     i8_linear8bit_backward_input,
     i8_linear8bit_forward,
+    i8_linear8bit_forward_multi,
     i8_linear8bit_forward_static,
     i8_linear8bit_matmul_dequant,
+    i8_linear8bit_multi_workspace_size,
     i8_linear8bit_prepare,
     i8_linear8bit_workspace_size,
     i8_outlier_columns,

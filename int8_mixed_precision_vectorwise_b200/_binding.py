@@ -33,6 +33,7 @@ EXPORTS = (
     "i8_int8_mm_dequant", "i8_dequant", "i8_linear8bit_workspace_size", "i8_linear8bit_forward",
     "i8_read_status", "i8_selftest_bounded_wait", "i8_linear8bit_prepare", "i8_linear8bit_matmul_dequant",
     "i8_linear8bit_forward_static", "i8_dequant_transposed", "i8_linear8bit_backward_input",
+    "i8_linear8bit_multi_workspace_size", "i8_linear8bit_forward_multi",
 )
 
 
@@ -61,6 +62,8 @@ def _declare(lib):
         "i8_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
         "i8_dequant_transposed": (_I, [_P, _P, _I, _I, _P, _P]),
         "i8_linear8bit_backward_input": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+        "i8_linear8bit_multi_workspace_size": (_S, [_I, _I, _I, _P, _I]),
+        "i8_linear8bit_forward_multi": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _F, _P, _S, _I, _P]),
         "i8_linear8bit_workspace_size": (_S, [_I, _I, _I, _I]),
         "i8_linear8bit_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
         "i8_linear8bit_prepare": (_I, [_P, _P, _I, _I, _I, _F, _P, _S, _I, _P]),
@@ -233,6 +236,48 @@ def i8_linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, out=Non
         _ptr(X), _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out),
         _ptr(workspace), workspace.numel(), max_outlier_cols, _stream(dev)))
     return out, workspace
+
+
+def _ptr_array(ts):
+    return (ctypes.c_void_p * len(ts))(*[None if t is None else t.data_ptr() for t in ts])
+
+
+def i8_linear8bit_multi_workspace_size(M: int, K: int, Ns, max_outlier_cols: int) -> int:
+    arr = (ctypes.c_int * len(Ns))(*Ns)
+    n = lib().i8_linear8bit_multi_workspace_size(M, K, len(Ns), arr, max_outlier_cols)
+    if n == 0:
+        raise I8Error("i8_linear8bit_multi_workspace_size", 1)
+    return int(n)
+
+
+def i8_linear8bit_forward_multi(X, CBs, SCBs, biases=None, threshold: float = 6.0, outs=None, workspace=None,
+                                max_outlier_cols: int = 256):
+    """Forward of several weights over the same X (X quantised once).  Returns (outs, workspace)."""
+    _need(X, torch.float16, "X", 2)
+    G = len(CBs)
+    if len(SCBs) != G or (biases is not None and len(biases) != G) or (outs is not None and len(outs) != G):
+        raise ValueError("CBs, SCBs, biases and outs must have one entry per weight")
+    biases = [None] * G if biases is None else list(biases)
+    M, K = X.shape
+    dev = X.device
+    for g in range(G):
+        _need(CBs[g], torch.int8, "CB", 2)
+        _need(SCBs[g], torch.float32, "SCB", 1)
+        if biases[g] is not None:
+            _need(biases[g], torch.float16, "bias", 1)
+        if CBs[g].shape[1] != K:
+            raise ValueError("X and every CB must share K")
+    Ns = [int(CB.shape[0]) for CB in CBs]
+    need = i8_linear8bit_multi_workspace_size(M, K, Ns, max_outlier_cols)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    if outs is None:
+        outs = [torch.empty((M, n), dtype=torch.float16, device=dev) for n in Ns]
+    n_arr = (ctypes.c_int * G)(*Ns)
+    _check("i8_linear8bit_forward_multi", lib().i8_linear8bit_forward_multi(
+        _ptr(X), M, K, G, _ptr_array(CBs), _ptr_array(SCBs), _ptr_array(biases), n_arr, _ptr_array(outs),
+        float(threshold), _ptr(workspace), workspace.numel(), max_outlier_cols, _stream(dev)))
+    return outs, workspace
 
 
 def i8_linear8bit_prepare(X, CB, threshold: float, workspace, max_outlier_cols: int = 256):

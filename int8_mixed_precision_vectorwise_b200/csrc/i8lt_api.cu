@@ -25,23 +25,43 @@ constexpr size_t kHdrBytes = 256;                      // status, used count, to
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+constexpr int kMaxGroups = 16;                        // weights per multi-weight forward
+
 struct WsLayout {
   size_t hdr, bitmap, counters, idx, sca, ca, xo, wo, partials, total;
   size_t clear_bytes;  // prefix cleared by every call: header, bitmap, split-K counters
   int ld_o;            // row stride (fp16 elements) of the gathered outlier operands
   bool decode;         // few tokens: the decode GEMM (split-K partials, no W_O gather)
+  int n_counters;      // split-K counters of all weights (decode)
 };
 
-bool ws_layout(int M, int N, int K, int cap, WsLayout* L) {
-  if (M <= 0 || N <= 0 || K <= 0 || cap < 0) return false;
+inline int decode_counters(int N) { return ((N + 127) / 128) * 4; }
+
+// Layout for G weights (N[g] output rows each) that read the same X [M, K]: the
+// quantised X, its outlier list and X[:, O] once; per weight its gathered
+// outlier rows W_O (more than 16 tokens) or its split-K counters (16 or fewer;
+// the partial-sum area is reused by the weights' GEMMs in turn).
+bool ws_layout_multi(int M, int K, int G, const int* N, int cap, WsLayout* L) {
+  if (M <= 0 || K <= 0 || cap < 0 || G < 1 || G > kMaxGroups || N == nullptr) return false;
+  for (int g = 0; g < G; ++g)
+    if (N[g] <= 0) return false;
   L->decode = M <= i8lt::kDecodeMaxTokens;
+  L->n_counters = 0;
+  size_t wo_bytes = 0, partial_bytes = 0;
+  for (int g = 0; g < G; ++g) {
+    L->n_counters += decode_counters(N[g]);
+    const size_t pb = static_cast<size_t>(i8lt::decode_slots(N[g], K)) * i8lt::kDecodeMaxTokens * N[g] * 8;
+    partial_bytes = pb > partial_bytes ? pb : partial_bytes;
+  }
+  L->ld_o = cap > 0 ? ((cap + 63) / 64) * 64 : 0;
+  for (int g = 0; g < G; ++g) wo_bytes += align256(static_cast<size_t>(N[g]) * L->ld_o * 2);
   size_t off = 0;
   L->hdr = off;
   off += kHdrBytes;
   L->bitmap = off;
   off += align256(static_cast<size_t>((K + 31) / 32) * 4);
   L->counters = off;
-  off += L->decode ? align256(static_cast<size_t>((N + 127) / 128) * 4 * 4) : 0;
+  off += L->decode ? align256(static_cast<size_t>(L->n_counters) * 4) : 0;
   L->clear_bytes = off;
   L->idx = off;
   off += align256(static_cast<size_t>(cap > 0 ? cap : 1) * 4);
@@ -49,16 +69,29 @@ bool ws_layout(int M, int N, int K, int cap, WsLayout* L) {
   off += align256(static_cast<size_t>(M) * 4);
   L->ca = off;
   off += align256(static_cast<size_t>(M) * K);
-  L->ld_o = cap > 0 ? ((cap + 63) / 64) * 64 : 0;
   L->xo = off;
   off += align256(static_cast<size_t>(M) * L->ld_o * 2);
   L->wo = off;
-  off += L->decode ? 0 : align256(static_cast<size_t>(N) * L->ld_o * 2);
+  off += L->decode ? 0 : wo_bytes;
   L->partials = off;
   // int32 partials, then fp32 partials of the outlier term
-  off += L->decode ? align256(static_cast<size_t>(i8lt::decode_slots(N, K)) * i8lt::kDecodeMaxTokens * N * 8) : 0;
+  off += L->decode ? align256(partial_bytes) : 0;
   L->total = off;
   return true;
+}
+
+bool ws_layout(int M, int N, int K, int cap, WsLayout* L) { return ws_layout_multi(M, K, 1, &N, cap, L); }
+
+// Byte offsets of weight g's gathered outlier rows and split-K counters.
+size_t wo_offset(const WsLayout& L, const int* N, int g) {
+  size_t off = L.wo;
+  for (int h = 0; h < g; ++h) off += align256(static_cast<size_t>(N[h]) * L.ld_o * 2);
+  return off;
+}
+size_t counters_offset(const WsLayout& L, const int* N, int g) {
+  size_t off = L.counters;
+  for (int h = 0; h < g; ++h) off += static_cast<size_t>(decode_counters(N[h])) * 4;
+  return off;
 }
 
 // --------------------------------------------------------------- driver entry point
@@ -222,10 +255,9 @@ i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int 
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
   if (L.decode) {
-    // one cluster launch writes everything the decode GEMM reads, header and counters included
-    const int n_counters = ((N + 127) / 128) * 4;
+    // one cluster launch writes everything the decode GEMMs read, header and counters included
     return cuda_status(i8lt::launch_decode_prep(Xh, M, K, threshold, cap, w.CA, w.SCA, w.idx,
-                                                cap > 0 ? w.XO : nullptr, L.ld_o, w.hdr, w.counters, n_counters,
+                                                cap > 0 ? w.XO : nullptr, L.ld_o, w.hdr, w.counters, L.n_counters,
                                                 st));
   }
   // status word, counts and bitmap are contiguous: one memset clears them
@@ -239,10 +271,11 @@ i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int 
                                                   (cap > 0 && !L.decode) ? w.WO : nullptr, L.ld_o, sms, st));
 }
 
-i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N, int K,
-                                 float threshold, i8_half* out, void* workspace, int cap, const WsLayout& L,
-                                 cudaStream_t st) {
-  const WsPtrs w = ws_ptrs(workspace, L);
+// The GEMM of one weight; `counters` / `WO` are that weight's split-K counters
+// (decode) or gathered outlier rows (prefill) in the workspace.
+i8_status enqueue_gemm(const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N, int K,
+                       float threshold, i8_half* out, const WsPtrs& w, int32_t* counters, __half* WO, int cap,
+                       const WsLayout& L, cudaStream_t st) {
   const bool with_o = threshold > 0.f && cap > 0;
   if (L.decode) {
     i8lt::DecodeArgs d{};
@@ -260,7 +293,7 @@ i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_ha
     d.ld_o = L.ld_o;
     d.partials = w.partials;
     d.slots = i8lt::decode_slots(N, K);
-    d.counters = w.counters;
+    d.counters = counters;
     d.status = w.hdr;
     d.wait_limit_ns = kWaitLimitNs;
     CUtensorMap tmW, tmC;
@@ -286,11 +319,18 @@ i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_ha
   a.n_used = with_o ? reinterpret_cast<const int32_t*>(w.hdr + 1) : nullptr;
   a.out_cap = cap;
   a.XO = with_o ? w.XO : nullptr;
-  a.WO = with_o ? w.WO : nullptr;
+  a.WO = with_o ? WO : nullptr;
   a.ld_o = L.ld_o;
   a.status = w.hdr;
   a.wait_limit_ns = kWaitLimitNs;
-  return run_gemm(w.CA, CB, M, N, K, a, false, with_o ? w.XO : nullptr, with_o ? w.WO : nullptr, L.ld_o, st);
+  return run_gemm(w.CA, CB, M, N, K, a, false, with_o ? w.XO : nullptr, with_o ? WO : nullptr, L.ld_o, st);
+}
+
+i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N, int K,
+                                 float threshold, i8_half* out, void* workspace, int cap, const WsLayout& L,
+                                 cudaStream_t st) {
+  const WsPtrs w = ws_ptrs(workspace, L);
+  return enqueue_gemm(CB, SCB, bias, M, N, K, threshold, out, w, w.counters, w.WO, cap, L, st);
 }
 
 }  // namespace
@@ -471,6 +511,54 @@ i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const float*
   s = enqueue_prepare(X, CB, M, N, K, threshold, workspace, max_outlier_cols, L, st);
   if (s != I8_OK) return s;
   return enqueue_matmul_dequant(CB, SCB, bias, M, N, K, threshold, out, workspace, max_outlier_cols, L, st);
+}
+
+size_t i8_linear8bit_multi_workspace_size(int M, int K, int G, const int* N, int max_outlier_cols) {
+  WsLayout L;
+  if (max_outlier_cols > kMaxOutlierCap || !ws_layout_multi(M, K, G, N, max_outlier_cols, &L)) return 0;
+  return L.total;
+}
+
+i8_status i8_linear8bit_forward_multi(const i8_half* X, int M, int K, int G, const int8_t* const* CB,
+                                      const float* const* SCB, const i8_half* const* bias, const int* N,
+                                      i8_half* const* out, float threshold, void* workspace, size_t workspace_bytes,
+                                      int max_outlier_cols, i8_stream_t stream) {
+  if (!X || !workspace || !CB || !SCB || !N || !out) return I8_ERR_INVALID_ARG;
+  if (G < 1 || G > kMaxGroups) return I8_ERR_INVALID_ARG;
+  const int cap = max_outlier_cols;
+  WsLayout L;
+  for (int g = 0; g < G; ++g) {
+    // every weight passes the single-weight checks against the same X and workspace rules
+    i8_status s = check_forward(X, CB[g], SCB[g], bias ? bias[g] : nullptr, M, N[g], K, threshold, out[g], true,
+                                workspace, ~size_t(0), cap, &L);
+    if (s != I8_OK) return s;
+  }
+  if (!ws_layout_multi(M, K, G, N, cap, &L)) return I8_ERR_INVALID_ARG;
+  if (workspace_bytes < L.total) return I8_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // X is quantised and its outlier columns found once; the first weight's
+  // outlier rows are gathered in the same launch
+  i8_status s = enqueue_prepare(X, CB[0], M, N[0], K, threshold, workspace, cap, L, st);
+  if (s != I8_OK) return s;
+  const WsPtrs w = ws_ptrs(workspace, L);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool gather_w = !L.decode && threshold > 0.f && cap > 0;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  for (int g = 0; g < G; ++g) {
+    __half* WO = reinterpret_cast<__half*>(ws + wo_offset(L, N, g));
+    int32_t* counters = reinterpret_cast<int32_t*>(ws + counters_offset(L, N, g));
+    if (g > 0 && gather_w) {
+      // this weight's outlier rows only: the list is rebuilt from the bitmap, X is not touched
+      s = cuda_status(i8lt::launch_outlier_prepare(w.bitmap, K, cap, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                                   nullptr, 0, nullptr, CB[g], N[g], WO, L.ld_o, sms, st));
+      if (s != I8_OK) return s;
+    }
+    s = enqueue_gemm(CB[g], SCB[g], bias ? bias[g] : nullptr, M, N[g], K, threshold, out[g], w, counters, WO, cap,
+                     L, st);
+    if (s != I8_OK) return s;
+  }
+  return I8_OK;
 }
 
 i8_status i8_read_status(const void* workspace, int32_t* count, i8_stream_t stream) {

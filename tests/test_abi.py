@@ -117,3 +117,37 @@ def test_backward_rejects(lib):
     assert g(FAKE, FAKE, 4, 12, 16, FAKE, None) == 2  # N % 8
     assert g(FAKE, FAKE_MIS, 4, 8, 16, FAKE, None) == 2
     assert lib.i8_read_status(None, None, None) == 1
+
+
+def test_multi_workspace_and_rejects(lib):
+    Ns = (ctypes.c_int * 3)(520, 264, 1040)
+    one = (ctypes.c_int * 1)(520)
+    f = lib.i8_linear8bit_multi_workspace_size
+    f.restype = ctypes.c_size_t
+    lib.i8_linear8bit_workspace_size.restype = ctypes.c_size_t
+    for M in (7, 300):   # few-token and prefill layouts
+        assert f(M, 1040, 1, one, 256) == lib.i8_linear8bit_workspace_size(M, 520, 1040, 256)
+        assert f(M, 1040, 3, Ns, 256) > f(M, 1040, 1, one, 256)
+    assert f(300, 1040, 0, Ns, 256) == 0
+    assert f(300, 1040, 17, Ns, 256) == 0
+    assert f(300, 1040, 3, None, 256) == 0
+    assert f(300, 1040, 3, (ctypes.c_int * 3)(520, 0, 8), 256) == 0
+    g = lib.i8_linear8bit_forward_multi
+    P3 = (ctypes.c_void_p * 3)(0x1000, 0x2000, 0x3000)
+    n = f(300, 1040, 3, Ns, 256)
+    ok = (FAKE, 300, 1040, 3, P3, P3, None, Ns, P3, ctypes.c_float(6.0), FAKE, ctypes.c_size_t(n), 256, None)
+
+    def call(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return g(*a)
+    assert call(a0=None) == 1                        # X
+    assert call(a3=0) == 1 and call(a3=17) == 1      # G
+    assert call(a4=None) == 1 and call(a7=None) == 1 and call(a8=None) == 1
+    assert call(a4=(ctypes.c_void_p * 3)(0x1000, None, 0x3000)) == 1   # a null weight
+    assert call(a2=1048) == 2                        # K % 16
+    assert call(a8=(ctypes.c_void_p * 3)(0x1000, 0x2008, 0x3000)) == 2  # misaligned output
+    assert call(a11=ctypes.c_size_t(n - 1)) == 3     # workspace too small
+    assert call(a9=ctypes.c_float(-1.0)) == 1
+

@@ -401,3 +401,61 @@ def test_backward_input_repeat_is_deterministic(i8):
     a = host(i8.i8_linear8bit_backward_input(dY, Wt))
     b = host(i8.i8_linear8bit_backward_input(dY, Wt))
     assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+# ------------------------------------------------------------------ several weights, one X
+MSHAPES = [
+    (300, 1040, (520, 264, 1040), 3, 6.0),    # prefill, few outlier columns
+    (512, 1024, (4096, 4096), 40, 6.0),       # prefill, > 16 columns: tcgen05 fp16 outlier path
+    (300, 1040, (520, 264), 3, 0.0),          # threshold 0
+    (7, 2064, (1000, 272, 4096), 5, 6.0),     # few tokens: one preparation, three decode GEMMs
+    (16, 4096, (4096, 1024), 40, 6.0),        # few tokens, many outlier columns
+]
+
+
+@pytest.mark.parametrize("M,K,Ns,n_out,tau", MSHAPES)
+def test_forward_multi_matches_single(i8, M, K, Ns, n_out, tau):
+    """Each output of the multi-weight forward is bit for bit the single forward of that
+    weight (same X), and within tolerance of the oracle."""
+    X, _ = act(M, K, n_out, seed=M + K + len(Ns))
+    dXd = dev(X)
+    ws_ref, CBs, SCBs, biases, host_w = [], [], [], [], []
+    for g, N in enumerate(Ns):
+        W = wl.weight(40 + g, N, K)
+        CB, SCB, _ = i8.i8_quantize_rowwise(dev(W), 0.0)
+        b = wl.bias(50 + g, N) if g % 2 == 0 else None
+        CBs.append(CB)
+        SCBs.append(SCB)
+        biases.append(None if b is None else dev(b))
+        host_w.append((W, b))
+    outs, ws = i8.i8_linear8bit_forward_multi(dXd, CBs, SCBs, biases, tau)
+    code, count = i8.i8_read_status(ws)
+    _, _, rcols = oracle.quantize_rowwise(X, tau)
+    assert code == 0
+    assert count == (len(rcols) if tau > 0 else 0)
+    for g in range(len(Ns)):
+        single, _ = i8.i8_linear8bit_forward(dXd, CBs[g], SCBs[g], biases[g], tau)
+        got = host(outs[g])
+        assert np.array_equal(got.view(np.uint16), host(single).view(np.uint16)), g
+        rCB, rSCB = oracle.quantize_weight_rowwise(host_w[g][0])
+        assert_close(got, oracle.linear8bit_forward(X, rCB, rSCB, host_w[g][1], tau), f"multi weight {g}")
+
+
+def test_forward_multi_reuses_workspace(i8):
+    """A second call on the same workspace with a different X (another outlier set) is correct:
+    the per-call state (status, counts, bitmap, split-K counters) is rebuilt each time."""
+    for M in (300, 9):
+        K, Ns = 1024, (768, 256)
+        W = [wl.weight(60 + g, N, K) for g, N in enumerate(Ns)]
+        CBs, SCBs = zip(*[i8.i8_quantize_rowwise(dev(w), 0.0)[:2] for w in W])
+        ws = torch.empty((i8.i8_linear8bit_multi_workspace_size(M, K, list(Ns), 256),), dtype=torch.uint8,
+                         device="cuda")
+        for seed, n_out in ((70, 6), (71, 2)):
+            X, _ = act(M, K, n_out, seed=seed)
+            outs, _ = i8.i8_linear8bit_forward_multi(dev(X), list(CBs), list(SCBs), None, 6.0, workspace=ws)
+            code, count = i8.i8_read_status(ws)
+            _, _, rcols = oracle.quantize_rowwise(X, 6.0)
+            assert (code, count) == (0, len(rcols))
+            for g in range(len(Ns)):
+                rCB, rSCB = oracle.quantize_weight_rowwise(W[g])
+                assert_close(host(outs[g]), oracle.linear8bit_forward(X, rCB, rSCB, None, 6.0), f"reuse {M} {g}")
