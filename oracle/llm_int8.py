@@ -1,4 +1,4 @@
-"""Plain CPU oracle for the LLM.int8() ``Linear8bitLt`` forward pass.
+"""Plain CPU oracle for the LLM.int8() ``Linear8bitLt`` forward pass and its input gradient.
 
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
 execute this module: only the test-suite, ``__graft_entry__.smoke()`` and the
@@ -36,7 +36,8 @@ listed with its reason in the design notes of the repository):
                    + (SCB[n]/127) * sum_{j in O} x[i,j]*CB[n,j] )``
       evaluated in float64 with one final round to fp16; the outlier weights
       are the int8 weights dequantised (the boundary takes no fp16 weight).
-* R7  input gradient (training through the frozen int8 layer):
+* R7  dequantize op: ``W = fp16(CB * SCB[n] / 127)``, one rounding.
+* R9  input gradient (training through the frozen int8 layer):
       ``dX = fp16(dY . W^)`` evaluated in float64 with one final round, where
       ``W^ = dequant(CB, SCB)`` is the fp16 dequantised weight.  This is the
       chain rule for ``y = X . W^T + bias``; the pages only say that int8
@@ -173,7 +174,7 @@ def int8_mm_dequant(C, SCA, SCB, bias=None) -> np.ndarray:
 
 
 def dequant(CB, SCB) -> np.ndarray:
-    """int8 dequantize op: ``W = fp16(CB * SCB[n] / 127)`` in float64.
+    """int8 dequantize op: ``W = fp16(CB * SCB[n] / 127)`` in float64 (reading R7).
 
     "LLM.int8() Refactoring: Part 1", section "Next steps"
     ("Add an int8 dequantize op").
@@ -227,7 +228,7 @@ def linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, rows=None)
 
 
 def linear8bit_backward_input(dY, CB, SCB, rows=None):
-    """Input gradient of the int8 linear layer (reading R7).
+    """Input gradient of the int8 linear layer (reading R9).
 
     "`bitsandbytes` - `Linear8bitLt` integration into `transformers` models",
     discussion of fine-tuning: trainable adapters sit on top of frozen int8
