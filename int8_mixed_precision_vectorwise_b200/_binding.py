@@ -119,16 +119,51 @@ def _need(t, dtype, name, ndim=None):
         raise ValueError(f"{name} must be {ndim}-D")
 
 
+def _check_shape(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check_device(t, dev, name):
+    if t.device != dev:
+        raise ValueError(f"{name} must be on {dev}, got {t.device}")
+
+
+def _arg(t, dtype, name, shape, dev):
+    """An input the kernels read: dtype, CUDA, contiguous, on `dev`, exactly `shape`."""
+    _need(t, dtype, name, len(shape))
+    _check_device(t, dev, name)
+    _check_shape(t, shape, name)
+    return t
+
+
+def _out(t, dtype, name, shape, dev):
+    """A caller-provided buffer the kernels write (checked like an input), or a new one."""
+    if t is None:
+        return torch.empty(tuple(shape), dtype=dtype, device=dev)
+    return _arg(t, dtype, name, shape, dev)
+
+
+def _workspace(t, dev, need):
+    """A caller workspace (uint8, on `dev`) large enough, else a new one."""
+    if t is not None:
+        _need(t, torch.uint8, "workspace", 1)
+        _check_device(t, dev, "workspace")
+        if t.numel() >= need:
+            return t
+    return torch.empty((need,), dtype=torch.uint8, device=dev)
+
+
 # ----------------------------------------------------------------- entry points
 def i8_quantize_rowwise(X, threshold: float = 0.0, CA=None, SCA=None, bitmap=None):
     """Fused row absmax + int8 quantisation + outlier bitmap.  Returns (CA, SCA, bitmap)."""
     _need(X, torch.float16, "X", 2)
     M, K = X.shape
     dev = X.device
-    CA = torch.empty((M, K), dtype=torch.int8, device=dev) if CA is None else CA
-    SCA = torch.empty((M,), dtype=torch.float32, device=dev) if SCA is None else SCA
-    if threshold > 0 and bitmap is None:
-        bitmap = torch.empty(((K + 31) // 32,), dtype=torch.int32, device=dev)
+    CA = _out(CA, torch.int8, "CA", (M, K), dev)
+    SCA = _out(SCA, torch.float32, "SCA", (M,), dev)
+    if threshold > 0 or bitmap is not None:
+        bitmap = _out(bitmap, torch.int32, "bitmap", ((K + 31) // 32,), dev)
     _check("i8_quantize_rowwise", lib().i8_quantize_rowwise(
         _ptr(X), M, K, float(threshold), _ptr(CA), _ptr(SCA), _ptr(bitmap), _stream(dev)))
     return CA, SCA, bitmap
@@ -138,8 +173,15 @@ def i8_outlier_columns(bitmap, K: int, max_cols: int, idx=None, count=None):
     """Sorted outlier column list from a bitmap.  Returns (idx[max_cols], count[1]) on device."""
     _need(bitmap, torch.int32, "bitmap", 1)
     dev = bitmap.device
-    idx = torch.empty((max(max_cols, 1),), dtype=torch.int32, device=dev) if idx is None else idx
-    count = torch.empty((1,), dtype=torch.int32, device=dev) if count is None else count
+    _check_shape(bitmap, ((K + 31) // 32,), "bitmap")
+    if idx is None:
+        idx = torch.empty((max(max_cols, 1),), dtype=torch.int32, device=dev)
+    else:
+        _need(idx, torch.int32, "idx", 1)
+        _check_device(idx, dev, "idx")
+        if idx.numel() < max_cols:
+            raise ValueError(f"idx must hold max_cols = {max_cols} entries")
+    count = _out(count, torch.int32, "count", (1,), dev)
     _check("i8_outlier_columns", lib().i8_outlier_columns(
         _ptr(bitmap), K, _ptr(idx), max_cols, _ptr(count), _stream(dev)))
     return idx, count
@@ -153,7 +195,8 @@ def i8_int8_linear_matmul(A, B, C=None):
     N = B.shape[0]
     if B.shape[1] != K:
         raise ValueError("A and B must share K")
-    C = torch.empty((M, N), dtype=torch.int32, device=A.device) if C is None else C
+    _check_device(B, A.device, "B")
+    C = _out(C, torch.int32, "C", (M, N), A.device)
     _check("i8_int8_linear_matmul", lib().i8_int8_linear_matmul(
         _ptr(A), _ptr(B), M, N, K, _ptr(C), _stream(A.device)))
     return C
@@ -162,12 +205,13 @@ def i8_int8_linear_matmul(A, B, C=None):
 def i8_int8_mm_dequant(C, SCA, SCB, bias=None, out=None):
     """out = fp16(C * SCA[i] * SCB[n] / 127^2 + bias[n])."""
     _need(C, torch.int32, "C", 2)
-    _need(SCA, torch.float32, "SCA", 1)
-    _need(SCB, torch.float32, "SCB", 1)
-    if bias is not None:
-        _need(bias, torch.float16, "bias", 1)
     M, N = C.shape
-    out = torch.empty((M, N), dtype=torch.float16, device=C.device) if out is None else out
+    dev = C.device
+    _arg(SCA, torch.float32, "SCA", (M,), dev)
+    _arg(SCB, torch.float32, "SCB", (N,), dev)
+    if bias is not None:
+        _arg(bias, torch.float16, "bias", (N,), dev)
+    out = _out(out, torch.float16, "out", (M, N), dev)
     _check("i8_int8_mm_dequant", lib().i8_int8_mm_dequant(
         _ptr(C), _ptr(SCA), _ptr(SCB), _ptr(bias), M, N, _ptr(out), _stream(C.device)))
     return out
@@ -176,9 +220,9 @@ def i8_int8_mm_dequant(C, SCA, SCB, bias=None, out=None):
 def i8_dequant(CB, SCB, W=None):
     """W = fp16(CB * SCB[n] / 127)."""
     _need(CB, torch.int8, "CB", 2)
-    _need(SCB, torch.float32, "SCB", 1)
     N, K = CB.shape
-    W = torch.empty((N, K), dtype=torch.float16, device=CB.device) if W is None else W
+    _arg(SCB, torch.float32, "SCB", (N,), CB.device)
+    W = _out(W, torch.float16, "W", (N, K), CB.device)
     _check("i8_dequant", lib().i8_dequant(_ptr(CB), _ptr(SCB), N, K, _ptr(W), _stream(CB.device)))
     return W
 
@@ -186,9 +230,9 @@ def i8_dequant(CB, SCB, W=None):
 def i8_dequant_transposed(CB, SCB, Wt=None):
     """Wt = W^T with W = fp16(CB * SCB[n] / 127): CB [N, K] -> Wt [K, N]."""
     _need(CB, torch.int8, "CB", 2)
-    _need(SCB, torch.float32, "SCB", 1)
     N, K = CB.shape
-    Wt = torch.empty((K, N), dtype=torch.float16, device=CB.device) if Wt is None else Wt
+    _arg(SCB, torch.float32, "SCB", (N,), CB.device)
+    Wt = _out(Wt, torch.float16, "Wt", (K, N), CB.device)
     _check("i8_dequant_transposed", lib().i8_dequant_transposed(
         _ptr(CB), _ptr(SCB), N, K, _ptr(Wt), _stream(CB.device)))
     return Wt
@@ -202,7 +246,8 @@ def i8_linear8bit_backward_input(dY, Wt, dX=None):
     K = Wt.shape[0]
     if Wt.shape[1] != N:
         raise ValueError("dY and Wt must share N")
-    dX = torch.empty((M, K), dtype=torch.float16, device=dY.device) if dX is None else dX
+    _check_device(Wt, dY.device, "Wt")
+    dX = _out(dX, torch.float16, "dX", (M, K), dY.device)
     _check("i8_linear8bit_backward_input", lib().i8_linear8bit_backward_input(
         _ptr(dY), _ptr(Wt), M, N, K, _ptr(dX), _stream(dY.device)))
     return dX
@@ -219,19 +264,16 @@ def i8_linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, out=Non
                           max_outlier_cols: int = 256):
     """LLM.int8() Linear8bitLt forward.  Returns (out, workspace)."""
     _need(X, torch.float16, "X", 2)
-    _need(CB, torch.int8, "CB", 2)
-    _need(SCB, torch.float32, "SCB", 1)
-    if bias is not None:
-        _need(bias, torch.float16, "bias", 1)
     M, K = X.shape
-    N = CB.shape[0]
-    if CB.shape[1] != K:
-        raise ValueError("X and CB must share K")
     dev = X.device
-    need = i8_linear8bit_workspace_size(M, N, K, max_outlier_cols)
-    if workspace is None or workspace.numel() < need:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
-    out = torch.empty((M, N), dtype=torch.float16, device=dev) if out is None else out
+    _need(CB, torch.int8, "CB", 2)
+    N = CB.shape[0]
+    _arg(CB, torch.int8, "CB", (N, K), dev)
+    _arg(SCB, torch.float32, "SCB", (N,), dev)
+    if bias is not None:
+        _arg(bias, torch.float16, "bias", (N,), dev)
+    workspace = _workspace(workspace, dev, i8_linear8bit_workspace_size(M, N, K, max_outlier_cols))
+    out = _out(out, torch.float16, "out", (M, N), dev)
     _check("i8_linear8bit_forward", lib().i8_linear8bit_forward(
         _ptr(X), _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out),
         _ptr(workspace), workspace.numel(), max_outlier_cols, _stream(dev)))
@@ -262,17 +304,14 @@ def i8_linear8bit_forward_multi(X, CBs, SCBs, biases=None, threshold: float = 6.
     dev = X.device
     for g in range(G):
         _need(CBs[g], torch.int8, "CB", 2)
-        _need(SCBs[g], torch.float32, "SCB", 1)
+        N = CBs[g].shape[0]
+        _arg(CBs[g], torch.int8, "CB", (N, K), dev)
+        _arg(SCBs[g], torch.float32, "SCB", (N,), dev)
         if biases[g] is not None:
-            _need(biases[g], torch.float16, "bias", 1)
-        if CBs[g].shape[1] != K:
-            raise ValueError("X and every CB must share K")
+            _arg(biases[g], torch.float16, "bias", (N,), dev)
     Ns = [int(CB.shape[0]) for CB in CBs]
-    need = i8_linear8bit_multi_workspace_size(M, K, Ns, max_outlier_cols)
-    if workspace is None or workspace.numel() < need:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
-    if outs is None:
-        outs = [torch.empty((M, n), dtype=torch.float16, device=dev) for n in Ns]
+    workspace = _workspace(workspace, dev, i8_linear8bit_multi_workspace_size(M, K, Ns, max_outlier_cols))
+    outs = [_out(None if outs is None else outs[g], torch.float16, "out", (M, Ns[g]), dev) for g in range(G)]
     n_arr = (ctypes.c_int * G)(*Ns)
     _check("i8_linear8bit_forward_multi", lib().i8_linear8bit_forward_multi(
         _ptr(X), M, K, G, _ptr_array(CBs), _ptr_array(SCBs), _ptr_array(biases), n_arr, _ptr_array(outs),
@@ -283,9 +322,12 @@ def i8_linear8bit_forward_multi(X, CBs, SCBs, biases=None, threshold: float = 6.
 def i8_linear8bit_prepare(X, CB, threshold: float, workspace, max_outlier_cols: int = 256):
     """First half of the forward: quantise X and prepare the outlier operands in `workspace`."""
     _need(X, torch.float16, "X", 2)
-    _need(CB, torch.int8, "CB", 2)
     M, K = X.shape
+    _need(CB, torch.int8, "CB", 2)
     N = CB.shape[0]
+    _arg(CB, torch.int8, "CB", (N, K), X.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check_device(workspace, X.device, "workspace")
     _check("i8_linear8bit_prepare", lib().i8_linear8bit_prepare(
         _ptr(X), _ptr(CB), M, N, K, float(threshold), _ptr(workspace), workspace.numel(),
         max_outlier_cols, _stream(X.device)))
@@ -296,6 +338,13 @@ def i8_linear8bit_matmul_dequant(CB, SCB, bias, M: int, threshold: float, out, w
     """Second half of the forward: the tensor-core GEMM with the fused epilogue."""
     _need(CB, torch.int8, "CB", 2)
     N, K = CB.shape
+    dev = CB.device
+    _arg(SCB, torch.float32, "SCB", (N,), dev)
+    if bias is not None:
+        _arg(bias, torch.float16, "bias", (N,), dev)
+    _arg(out, torch.float16, "out", (M, N), dev)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check_device(workspace, dev, "workspace")
     _check("i8_linear8bit_matmul_dequant", lib().i8_linear8bit_matmul_dequant(
         _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out), _ptr(workspace),
         workspace.numel(), max_outlier_cols, _stream(CB.device)))
@@ -306,13 +355,20 @@ def i8_linear8bit_forward_static(X, CB, SCB, bias=None, threshold: float = 6.0, 
                                  max_outlier_cols: int = 256, status_out=None):
     """Forward using the library's built-in scratch instead of a workspace (see include/i8lt.h)."""
     _need(X, torch.float16, "X", 2)
-    _need(CB, torch.int8, "CB", 2)
-    _need(SCB, torch.float32, "SCB", 1)
-    if bias is not None:
-        _need(bias, torch.float16, "bias", 1)
     M, K = X.shape
+    dev = X.device
+    _need(CB, torch.int8, "CB", 2)
     N = CB.shape[0]
-    out = torch.empty((M, N), dtype=torch.float16, device=X.device) if out is None else out
+    _arg(CB, torch.int8, "CB", (N, K), dev)
+    _arg(SCB, torch.float32, "SCB", (N,), dev)
+    if bias is not None:
+        _arg(bias, torch.float16, "bias", (N,), dev)
+    out = _out(out, torch.float16, "out", (M, N), dev)
+    if status_out is not None:
+        _need(status_out, torch.int32, "status_out", 1)
+        _check_device(status_out, dev, "status_out")
+        if status_out.numel() < 3:
+            raise ValueError("status_out must hold 3 words")
     _check("i8_linear8bit_forward_static", lib().i8_linear8bit_forward_static(
         _ptr(X), _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out), max_outlier_cols,
         _ptr(status_out), _stream(X.device)))

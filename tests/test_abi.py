@@ -151,3 +151,23 @@ def test_multi_workspace_and_rejects(lib):
     assert call(a11=ctypes.c_size_t(n - 1)) == 3     # workspace too small
     assert call(a9=ctypes.c_float(-1.0)) == 1
 
+
+
+def test_binding_shape_and_device_checks():
+    """The binding's buffer checks (shapes, devices, workspace reuse), exercised on CPU tensors:
+    the same helpers guard every entry point before a pointer reaches the library."""
+    import torch
+    from int8_mixed_precision_vectorwise_b200 import _binding as b
+    t = torch.zeros((3, 4), dtype=torch.float16)
+    b._check_shape(t, (3, 4), "t")
+    with pytest.raises(ValueError, match="shape"):
+        b._check_shape(t, (4, 3), "t")
+    with pytest.raises(ValueError, match="shape"):
+        b._check_shape(torch.zeros(12), (3, 4), "t")
+    b._check_device(t, torch.device("cpu"), "t")
+    with pytest.raises(ValueError, match="must be on"):
+        b._check_device(t, torch.device("cuda", 0), "t")
+    with pytest.raises(ValueError, match="CUDA"):
+        b._arg(t, torch.float16, "t", (3, 4), torch.device("cpu"))       # inputs must live on the GPU
+    with pytest.raises(TypeError, match="float16"):
+        b._arg(t.float(), torch.float16, "t", (3, 4), torch.device("cpu"))
