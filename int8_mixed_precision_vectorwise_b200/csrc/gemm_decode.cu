@@ -29,6 +29,8 @@
 // 72 KB stages keeps ~216 KB of weights in flight per SM.
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -434,12 +436,15 @@ __global__ void __launch_bounds__(DTHREADS, 1)
 template <int C>
 static cudaError_t launch_decode_c(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
                                    cudaStream_t st) {
-  static bool attr_done = false;
-  if (!attr_done) {
+  // the shared-memory opt-in, once per device (calls may come from several host threads)
+  static std::atomic<bool> attr_done[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm_i8_decode<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          DecodeCfg<C>::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
