@@ -54,6 +54,13 @@ def test_dequant_closed_form(case):
     assert W.astype(np.float64).tolist() == case["W"]
 
 
+@pytest.mark.parametrize("case", GOLD["backward"], ids=lambda c: c["name"])
+def test_backward_input_closed_form(case):
+    dX = oracle.linear8bit_backward_input(f16(case["dY"]), np.array(case["CB"], np.int8), np.float32(case["SCB"]))
+    assert dX.dtype == np.float16
+    assert dX.tolist() == case["dX"]
+
+
 @pytest.mark.parametrize("case", GOLD["forward"], ids=lambda c: c["name"])
 def test_forward_closed_form(case):
     out = oracle.linear8bit_forward(f16(case["X"]), np.array(case["CB"], np.int8),
