@@ -164,6 +164,12 @@ def job_throughput(ops_per_step: float, steps: int, world: int, ms: float) -> fl
     return world * ops_per_step * steps / (ms / 1e3) / 1e12
 
 
+def nearest_rank(xs, ps):
+    """Nearest-rank percentiles (p in [0, 1]) of a non-empty sample."""
+    v = sorted(xs)
+    return [v[min(len(v) - 1, max(0, int(round(p * (len(v) - 1)))))] for p in ps]
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def cpu_oracle_steps(layers_np, rows: int, steps: int, min_seconds: float = 0.0):
     """Run the oracle forward on the first `rows` rows of every linear; returns (seconds per step, ops per step)."""
@@ -582,7 +588,8 @@ def run_ours(args):
         barrier()
     ms = e0.elapsed_time(e1)
     ms_instr = g0.elapsed_time(g1)
-    gemm_ms = sum(a.elapsed_time(b) for row in ev for a, b in row)
+    gemm_step_ms = [sum(a.elapsed_time(b) for a, b in row) for row in ev]
+    gemm_ms = sum(gemm_step_ms)
     ms_max = max_over_ranks(ms, world, dist, dev)
 
     # ---- the same step with the inputs shared as in a decoder layer (informational)
@@ -727,6 +734,7 @@ def run_ours(args):
                      "unit": "TOPS", "frac": achieved / peak, "traffic": read_traffic(),
                      "peak_source": peak_src, "frac_of_other_peak": achieved / other,
                      "gemm_ms_per_step": gemm_ms / K, "gemm_share_of_step": gemm_ms / ms_instr,
+                     "gemm_ms_per_step_p10_p50_p90": nearest_rank(gemm_step_ms, (0.1, 0.5, 0.9)),
                      "gemm_timing": "CUDA events around each GEMM launch in a second pass of the same "
                                     f"{K} steps ({ms_instr / K:.4f} ms per instrumented step)"},
         "cpu_baseline": cpu,

@@ -64,6 +64,14 @@ def test_job_throughput_single_rank():
     assert bench.job_throughput(2e12, 10, 1, 1000.0) == pytest.approx(20.0)
 
 
+def test_nearest_rank_percentiles():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.nearest_rank([3.0], (0.1, 0.5, 0.9)) == [3.0, 3.0, 3.0]
+    xs = [float(x) for x in range(11, 0, -1)]          # 11 .. 1, unsorted input
+    assert bench.nearest_rank(xs, (0.0, 0.1, 0.5, 0.9, 1.0)) == [1.0, 2.0, 6.0, 10.0, 11.0]
+
+
 def test_reference_arm_reports_on_rank_zero_only():
     """Under torchrun every rank runs bench.py; the reference arm (the CPU oracle) runs and
     prints on rank 0 alone and the other ranks exit 0 without work."""
