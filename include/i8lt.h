@@ -1,5 +1,6 @@
 /*
- * i8lt.h — C ABI of the B200 (sm_100a) LLM.int8() Linear8bitLt forward library.
+ * i8lt.h — C ABI of the B200 (sm_100a) LLM.int8() Linear8bitLt forward library
+ * (with the input gradient through a frozen int8 layer).
  *
  * The operation is the mixed int8/fp16 decomposition of
  * "`bitsandbytes` - `Linear8bitLt` integration into `transformers` models"
@@ -24,7 +25,8 @@
  *     kernels enqueued".  Nothing synchronises the host except i8_read_status.
  *   - Argument errors are returned before anything is enqueued.  Matrix
  *     pointers must be 16-byte aligned and K must be a multiple of 16 (the TMA
- *     row-stride rule); M, N, K must be > 0.  The threshold must be finite and
+ *     row-stride rule; the gradient entry points state their own rule); M, N,
+ *     K must be > 0.  The threshold must be finite and
  *     >= 0; 0 turns outlier handling off.
  *   - Errors found on the device (more outlier columns than the workspace
  *     holds, a pipeline wait that ran past its time limit) are written to a
