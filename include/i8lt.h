@@ -20,6 +20,8 @@
  *     owns every buffer: the library never allocates or frees memory, keeps no
  *     mutable global state, and may be called concurrently on different
  *     streams as long as the calls do not share output or workspace buffers.
+ *     The one exception is i8_linear8bit_forward_static, whose calls share one
+ *     scratch array built into the library (see its note).
  *   - All work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream) and is asynchronous: I8_OK means "arguments valid and
  *     kernels enqueued".  Nothing synchronises the host except i8_read_status.
@@ -110,6 +112,26 @@ I8_API i8_status i8_int8_linear_matmul(const int8_t* A, const int8_t* B, int M, 
                                 int32_t* C, i8_stream_t stream);
 
 /*
+ * i8_int8_linear_matmul_ws — the same exact product, C = A . B^T in int32,
+ * computed by the kernel the forward itself uses for these sizes: for
+ * M <= 16 rows the few-token stream-K kernel (its k-range split across CTAs,
+ * partial sums combined in the workspace), for more rows the tensor-core
+ * GEMM of i8_int8_linear_matmul.  It lets a caller check that few-token
+ * kernel's integer sums on their own, before any scaling.
+ *   workspace: device memory, 256-byte aligned, of at least
+ *     i8_int8_linear_matmul_workspace_size(M, N, K) bytes (0 for M > 16:
+ *     NULL is then accepted).  Its contents on entry do not matter.
+ *   status: optional device uint32 (NULL to skip).  The call first sets it to
+ *     I8_OK, in stream order; a pipeline wait that ran past its time limit
+ *     then sets it to I8_ERR_TIMEOUT (C is unspecified in that case).
+ * Same operand rules as i8_int8_linear_matmul.
+ */
+I8_API size_t i8_int8_linear_matmul_workspace_size(int M, int N, int K);
+I8_API i8_status i8_int8_linear_matmul_ws(const int8_t* A, const int8_t* B, int M, int N, int K, int32_t* C,
+                                          void* workspace, size_t workspace_bytes, uint32_t* status,
+                                          i8_stream_t stream);
+
+/*
  * i8_int8_mm_dequant — out = fp16(C * SCA[i] * SCB[n] / 127^2 + bias[n])
  * ("LLM.int8() Refactoring: Part 1", section "Deprecations": mm_dequant
  * becomes int8_mm_dequant; commit "New naive mm_dequant kernel for row-major").
@@ -139,6 +161,21 @@ I8_API i8_status i8_dequant_transposed(const int8_t* CB, const float* SCB, int N
                                 i8_half* Wt, i8_stream_t stream);
 
 /*
+ * i8_gather_column_blocks — the output of a layer split by output columns
+ * over P GPUs ("column parallel": the exllama issue #95 discussion of tensor
+ * parallelism splits a linear layer's weight between GPUs; the
+ * `Linear8bitLt` integration page spreads BLOOM-176B's int8 weights over
+ * several A100s).  Rank p holds rows [p*Np, (p+1)*Np) of CB / SCB / bias and
+ * computes out_p [M, Np] on the replicated X; an all-gather of the out_p
+ * leaves them rank-major in G [P, M, Np] (each block contiguous); this puts
+ * them in place:
+ *   out[m, p*Np + j] = G[p, m, j],   out [M, P*Np] fp16, row-major.
+ * A plain copy (bit for bit).  G and out 16-byte aligned, P*Np < 2^31.
+ */
+I8_API i8_status i8_gather_column_blocks(const i8_half* G, int P, int M, int Np, i8_half* out,
+                                         i8_stream_t stream);
+
+/*
  * i8_linear8bit_backward_input — input gradient of the int8 linear layer:
  *   dX[i, k] = fp16( sum_n dY[i, n] * Wt[k, n] ),  fp32 accumulation,
  * i.e. dX = dY . W^ for y = X . W^T + bias with W^ = Wt^T.  With Wt from
@@ -151,10 +188,21 @@ I8_API i8_status i8_dequant_transposed(const int8_t* CB, const float* SCB, int N
  * runs on the tensor cores in fp16 (tcgen05 kind::f16).
  *   dY [M, N] fp16, Wt [K, N] fp16, dX [M, K] fp16 output.
  * Requires N % 8 == 0 (16-byte rows of dY and Wt).  A pipeline wait that ran
- * past its time limit leaves dX unspecified and is not reported.
+ * past its time limit leaves dX unspecified; this entry point does not report
+ * it, i8_linear8bit_backward_input_status does.
  */
 I8_API i8_status i8_linear8bit_backward_input(const i8_half* dY, const i8_half* Wt, int M, int N,
                                        int K, i8_half* dX, i8_stream_t stream);
+
+/*
+ * The same input gradient with a status word: `status` (device uint32, 4-byte
+ * aligned, or NULL) is set to I8_OK first, in stream order, and to
+ * I8_ERR_TIMEOUT if a pipeline wait ran past its time limit (dX is then
+ * unspecified).
+ */
+I8_API i8_status i8_linear8bit_backward_input_status(const i8_half* dY, const i8_half* Wt, int M, int N,
+                                                     int K, i8_half* dX, uint32_t* status,
+                                                     i8_stream_t stream);
 
 /*
  * Workspace bytes i8_linear8bit_forward needs for these sizes.  The workspace
@@ -163,6 +211,36 @@ I8_API i8_status i8_linear8bit_backward_input(const i8_half* dY, const i8_half* 
  * status word.  Returns 0 for invalid sizes.
  */
 I8_API size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_cols);
+
+/*
+ * Where i8_linear8bit_prepare leaves its results inside the workspace (byte
+ * offsets from its start), so that a caller can read the prepared operands
+ * back: after i8_linear8bit_prepare (or a whole forward) has run,
+ *   header  uint32 [3]: status word, outlier columns gathered (used = min(total,
+ *           max_outlier_cols)), outlier columns found (total);
+ *   bitmap  uint32 [ceil(K/32)] outlier-column bitmap (M > 16 only; for M <= 16
+ *           the preparation keeps it on chip and this region is unused);
+ *   idx     int32 [used]: the outlier columns, ascending (the state.idx of
+ *           "LLM.int8() Refactoring: Part 1", review of _functions.py);
+ *   sca     fp32 [M] row scales; ca  int8 [M, K] codes, 0 in every outlier column;
+ *   x_o     fp16 [M, ld_o] gathered X[:, idx]; w_o  fp16 [N, ld_o] gathered
+ *           fp16(CB[:, idx]) (M > 16 only).
+ * Order of the gathered columns: for M > 16, within each group of 16 list
+ * entries the stored positions hold entries (0 1 8 9)(2 3 10 11)(4 5 12 13)
+ * (6 7 14 15) of the group, i.e. position p holds entry
+ * 16*(p/16) + 2*((p%16)/4) + (p%2) + 8*((p%4)/2) (the order of an m16n8k16
+ * operand fragment), and positions past `used` up to the next multiple of 64
+ * (16 when used <= 16) are 0.  For M <= 16, x_o holds the entries in list
+ * order, zero up to the next multiple of 16.
+ * few_tokens is 1 when M <= 16 (the few-token kernels are used).
+ */
+typedef struct {
+  size_t header, bitmap, idx, sca, ca, x_o, w_o, total;
+  int ld_o;
+  int few_tokens;
+} i8_workspace_layout;
+I8_API i8_status i8_linear8bit_workspace_layout(int M, int N, int K, int max_outlier_cols,
+                                                i8_workspace_layout* layout);
 
 /*
  * i8_linear8bit_forward — LLM.int8() Linear8bitLt forward
@@ -272,7 +350,11 @@ I8_API i8_status i8_read_status(const void* workspace, int32_t* count, i8_stream
  * Sizes whose workspace (i8_linear8bit_workspace_size) exceeds 32 MiB are
  * rejected with I8_ERR_WORKSPACE before anything is enqueued.
  * The first call on each device looks up the array's device address and must
- * happen before any stream capture that records this call.  All calls share
+ * happen before any stream capture that records this call.  The address is
+ * kept per device and CUDA context: if the device's context is destroyed and
+ * created again (cudaDeviceReset, or a framework that tears its context
+ * down), the next call looks the array up again, so that call too must come
+ * before any stream capture.  All calls share
  * the one array and it keeps the previous call's contents (each call clears
  * what must start at zero), so calls that can overlap on the GPU — on two
  * streams, or from two host threads — race; serialise them on one stream.

@@ -11,7 +11,9 @@ from ._binding import (  # noqa: F401
     STATUS,
     i8_dequant,
     i8_dequant_transposed,
+    i8_gather_column_blocks,
     i8_int8_linear_matmul,
+    i8_int8_linear_matmul_ws,
     i8_int8_mm_dequant,
     i8_linear8bit_backward_input,
     i8_linear8bit_forward,
@@ -20,6 +22,7 @@ from ._binding import (  # noqa: F401
     i8_linear8bit_matmul_dequant,
     i8_linear8bit_multi_workspace_size,
     i8_linear8bit_prepare,
+    i8_linear8bit_workspace_layout,
     i8_linear8bit_workspace_size,
     i8_outlier_columns,
     i8_quantize_rowwise,

@@ -34,7 +34,17 @@ EXPORTS = (
     "i8_read_status", "i8_selftest_bounded_wait", "i8_linear8bit_prepare", "i8_linear8bit_matmul_dequant",
     "i8_linear8bit_forward_static", "i8_dequant_transposed", "i8_linear8bit_backward_input",
     "i8_linear8bit_multi_workspace_size", "i8_linear8bit_forward_multi",
+    "i8_int8_linear_matmul_workspace_size", "i8_int8_linear_matmul_ws", "i8_linear8bit_workspace_layout",
+    "i8_linear8bit_backward_input_status", "i8_gather_column_blocks",
 )
+
+
+class WorkspaceLayout(ctypes.Structure):
+    """Mirror of ``i8_workspace_layout`` (byte offsets into a forward workspace)."""
+    _fields_ = [("header", ctypes.c_size_t), ("bitmap", ctypes.c_size_t), ("idx", ctypes.c_size_t),
+                ("sca", ctypes.c_size_t), ("ca", ctypes.c_size_t), ("x_o", ctypes.c_size_t),
+                ("w_o", ctypes.c_size_t), ("total", ctypes.c_size_t), ("ld_o", ctypes.c_int),
+                ("few_tokens", ctypes.c_int)]
 
 
 class I8Error(RuntimeError):
@@ -61,6 +71,7 @@ def _declare(lib):
         "i8_int8_mm_dequant": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
         "i8_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
         "i8_dequant_transposed": (_I, [_P, _P, _I, _I, _P, _P]),
+        "i8_gather_column_blocks": (_I, [_P, _I, _I, _I, _P, _P]),
         "i8_linear8bit_backward_input": (_I, [_P, _P, _I, _I, _I, _P, _P]),
         "i8_linear8bit_multi_workspace_size": (_S, [_I, _I, _I, _P, _I]),
         "i8_linear8bit_forward_multi": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _F, _P, _S, _I, _P]),
@@ -70,6 +81,10 @@ def _declare(lib):
         "i8_linear8bit_matmul_dequant": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P, _S, _I, _P]),
         "i8_linear8bit_forward_static": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P]),
         "i8_read_status": (_I, [_P, _P, _P]),
+        "i8_int8_linear_matmul_workspace_size": (_S, [_I, _I, _I]),
+        "i8_int8_linear_matmul_ws": (_I, [_P, _P, _I, _I, _I, _P, _P, _S, _P, _P]),
+        "i8_linear8bit_workspace_layout": (_I, [_I, _I, _I, _I, ctypes.POINTER(WorkspaceLayout)]),
+        "i8_linear8bit_backward_input_status": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
         "i8_selftest_bounded_wait": (_I, [_P, ctypes.c_uint64, _P]),
     }
     for name, (res, args) in sig.items():
@@ -202,6 +217,37 @@ def i8_int8_linear_matmul(A, B, C=None):
     return C
 
 
+def i8_int8_linear_matmul_ws(A, B, C=None, workspace=None, status=None):
+    """C = A . B^T (int32, exact) by the kernel the forward uses for these sizes: for at
+    most 16 rows of A the few-token stream-K kernel, whose split-K partial sums live in
+    `workspace` (allocated here when None).  `status` (int32 [1] on the device, optional)
+    receives the device status word.  Returns (C, workspace)."""
+    _need(A, torch.int8, "A", 2)
+    _need(B, torch.int8, "B", 2)
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("A and B must share K")
+    dev = A.device
+    _check_device(B, dev, "B")
+    C = _out(C, torch.int32, "C", (M, N), dev)
+    need = int(lib().i8_int8_linear_matmul_workspace_size(M, N, K))
+    workspace = _workspace(workspace, dev, max(need, 1))
+    if status is not None:
+        _arg(status, torch.int32, "status", (1,), dev)
+    _check("i8_int8_linear_matmul_ws", lib().i8_int8_linear_matmul_ws(
+        _ptr(A), _ptr(B), M, N, K, _ptr(C), _ptr(workspace), workspace.numel(), _ptr(status), _stream(dev)))
+    return C, workspace
+
+
+def i8_linear8bit_workspace_layout(M: int, N: int, K: int, max_outlier_cols: int) -> dict:
+    """Byte offsets of the prepared operands inside a forward workspace (see include/i8lt.h)."""
+    lay = WorkspaceLayout()
+    _check("i8_linear8bit_workspace_layout",
+           lib().i8_linear8bit_workspace_layout(M, N, K, max_outlier_cols, ctypes.byref(lay)))
+    return {name: int(getattr(lay, name)) for name, _ in WorkspaceLayout._fields_}
+
+
 def i8_int8_mm_dequant(C, SCA, SCB, bias=None, out=None):
     """out = fp16(C * SCA[i] * SCB[n] / 127^2 + bias[n])."""
     _need(C, torch.int32, "C", 2)
@@ -238,8 +284,19 @@ def i8_dequant_transposed(CB, SCB, Wt=None):
     return Wt
 
 
-def i8_linear8bit_backward_input(dY, Wt, dX=None):
-    """dX = fp16(dY . Wt^T): dY [M, N], Wt [K, N] (from i8_dequant_transposed) -> dX [M, K]."""
+def i8_gather_column_blocks(G, out=None):
+    """out [M, P*Np] from rank-major column blocks G [P, M, Np]: out[m, p*Np + j] = G[p, m, j]."""
+    _need(G, torch.float16, "G", 3)
+    P, M, Np = G.shape
+    out = _out(out, torch.float16, "out", (M, P * Np), G.device)
+    _check("i8_gather_column_blocks", lib().i8_gather_column_blocks(
+        _ptr(G), P, M, Np, _ptr(out), _stream(G.device)))
+    return out
+
+
+def i8_linear8bit_backward_input(dY, Wt, dX=None, status=None):
+    """dX = fp16(dY . Wt^T): dY [M, N], Wt [K, N] (from i8_dequant_transposed) -> dX [M, K].
+    `status` (int32 [1] on the device, optional) receives the device status word."""
     _need(dY, torch.float16, "dY", 2)
     _need(Wt, torch.float16, "Wt", 2)
     M, N = dY.shape
@@ -248,8 +305,13 @@ def i8_linear8bit_backward_input(dY, Wt, dX=None):
         raise ValueError("dY and Wt must share N")
     _check_device(Wt, dY.device, "Wt")
     dX = _out(dX, torch.float16, "dX", (M, K), dY.device)
-    _check("i8_linear8bit_backward_input", lib().i8_linear8bit_backward_input(
-        _ptr(dY), _ptr(Wt), M, N, K, _ptr(dX), _stream(dY.device)))
+    if status is None:
+        _check("i8_linear8bit_backward_input", lib().i8_linear8bit_backward_input(
+            _ptr(dY), _ptr(Wt), M, N, K, _ptr(dX), _stream(dY.device)))
+    else:
+        _arg(status, torch.int32, "status", (1,), dY.device)
+        _check("i8_linear8bit_backward_input_status", lib().i8_linear8bit_backward_input_status(
+            _ptr(dY), _ptr(Wt), M, N, K, _ptr(dX), _ptr(status), _stream(dY.device)))
     return dX
 
 

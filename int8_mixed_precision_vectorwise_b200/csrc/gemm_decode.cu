@@ -330,6 +330,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
     const int quad = warp & 3;  // TMEM lanes = weight rows quad*32 .. +31 of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     pdl_wait();  // scales and the outlier count come from the preceding kernel
+    const bool raw = p.C != nullptr;  // store the int32 sums instead of the dequantised outputs
     const int n_used = p.n_used != nullptr ? min(max(*p.n_used, 0), p.out_cap) : 0;
     const size_t dpart = static_cast<size_t>(p.slots) * DT * N;  // fp32 partials follow the int32 ones
     int it = 0;
@@ -339,8 +340,8 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       const int n = tile * DM + quad * 32 + lane;
-      const float sb = n < N ? __ldg(p.SCB + n) : 0.f;
-      const float bv = (n < N && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
+      const float sb = (!raw && n < N) ? __ldg(p.SCB + n) : 0.f;
+      const float bv = (!raw && n < N && p.bias != nullptr) ? __half2float(p.bias[n]) : 0.f;
       int ok = 0;
       if (lane == 0) ok = mbar_wait_bounded(&acc_full[buf], use & 1u, s_abort, p.status, p.wait_limit_ns) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -414,6 +415,15 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         }
       }
       if (!finalize || n >= N) continue;
+      if (raw) {
+        // the exact int32 sums C[t, n], t < T (lanes write consecutive n)
+#pragma unroll
+        for (int t = 0; t < DT; ++t) {
+          if (t >= T) break;
+          p.C[static_cast<size_t>(t) * N + n] = static_cast<int32_t>(c[t]);
+        }
+        continue;
+      }
       // dequant + bias + outlier term for (t, n), t < T
 #pragma unroll
       for (int t = 0; t < DT; ++t) {
@@ -435,7 +445,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
 
 template <int C>
 static cudaError_t launch_decode_c(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
-                                   cudaStream_t st) {
+                                   bool pdl, cudaStream_t st) {
   // the shared-memory opt-in, once per device (calls may come from several host threads)
   static std::atomic<bool> attr_done[64];
   int dev = 0;
@@ -455,16 +465,16 @@ static cudaError_t launch_decode_c(const CUtensorMap& tmW, const CUtensorMap& tm
   attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr.val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = &attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k_gemm_i8_decode<C>, tmW, tmC, a);
 }
 
 cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
-                               int boxes_per_stage, cudaStream_t st) {
+                               int boxes_per_stage, bool pdl, cudaStream_t st) {
   switch (boxes_per_stage) {
-    case 2: return launch_decode_c<2>(tmW, tmC, a, grid, st);
-    case 4: return launch_decode_c<4>(tmW, tmC, a, grid, st);
-    default: return launch_decode_c<1>(tmW, tmC, a, grid, st);
+    case 2: return launch_decode_c<2>(tmW, tmC, a, grid, pdl, st);
+    case 4: return launch_decode_c<4>(tmW, tmC, a, grid, pdl, st);
+    default: return launch_decode_c<1>(tmW, tmC, a, grid, pdl, st);
   }
 }
 

@@ -2,7 +2,7 @@
 // LLM.int8() dequant epilogue fused in.
 //
 //   C[i, n]  = sum_k CA[i, k] * CB[n, k]                       (tcgen05 kind::i8, int32 in TMEM)
-//   D[i, n]  = sum_{j in O} X[i, j] * CB[n, j]                  (tcgen05 kind::f16, fp32 in TMEM)
+//   D[i, n]  = sum_{j in O} X[i, j] * CB[n, j]                  (warp MMAs, or tcgen05 kind::f16)
 //   out      = fp16(C * SCA[i] * SCB[n] / 127^2 + bias[n] + D * SCB[n] / 127)
 //
 // which is the mixed decomposition of "`bitsandbytes` - `Linear8bitLt`
@@ -25,13 +25,16 @@
 // in the leader, issues tcgen05.mma (one lane); warps 2-9 run the epilogue
 // (two warps per 32-lane TMEM quadrant, one per 128-column half).  K streams
 // through a 6-stage ring of 128-byte-deep, 128B-swizzled tiles; the gathered
-// fp16 outlier tiles (64 fp16 = 128 bytes deep) use the same ring after the
-// int8 k-blocks.  TMEM: 512 columns.  Two 256-column int32 accumulators
-// alternate so the epilogue of tile t overlaps the mainloop of tile t+1.  Up
-// to 16 outlier columns, the epilogue adds the (rank <= 16) outlier product
-// itself with warp-level MMAs (mma.sync m16n8k16) on the gathered operands;
-// with more, tcgen05 kind::f16 MMAs write D into TMEM columns [256,512) and
-// the accumulator is single-buffered.
+// fp16 outlier tiles (64 fp16 = 128 bytes deep) use the same ring.  TMEM: 512
+// columns.  Two 256-column accumulators alternate so the epilogue of tile t
+// overlaps the mainloop of tile t+1.  Up to 16 outlier columns, the epilogue
+// adds the (rank <= 16) outlier product itself with warp-level MMAs
+// (mma.sync m16n8k16) on the gathered operands.  With more, the epilogue
+// first rewrites tile t's int32 accumulator in place as fp32 C * SCA / 127
+// (tcgen05.ld, convert, tcgen05.st) and the MMA thread adds tcgen05 kind::f16
+// MMAs of the outlier tiles on top of it; it issues them a few k-blocks into
+// tile t+1's mainloop, so the tensor pipe does not wait for the conversion.
+// The epilogue then scales by SCB / 127 and adds the bias.
 // The epilogue writes fp16 32x32 boxes through shared memory with TMA stores.
 //
 // A third mode runs the same pipeline as a plain fp16 GEMM, out = fp16(XO . WO^T)
@@ -40,6 +43,8 @@
 // input gradient dX = dY . W^ of a linear layer whose frozen weight W^ is the
 // dequantised int8 weight, with XO = dY [M, N] and WO = W^ transposed [K, N].
 #include <cuda_fp16.h>
+
+#include <atomic>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -63,7 +68,7 @@ constexpr int OBOX = kGemmOutBox;                // 32 x 32 fp16 output box
 constexpr int STG_BYTES = OBOX * OBOX * 2;       // 2 KB
 constexpr int STG_OFF = RING_BYTES;
 constexpr int STG_TOTAL = EPI_WARPS * 2 * STG_BYTES;
-constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int NUM_BARS = 2 * STAGES + 9;
 constexpr int BAR_OFF = STG_OFF + STG_TOTAL;
 constexpr int MISC_OFF = BAR_OFF + ((NUM_BARS * 8 + 15) / 16) * 16;
 constexpr int SMEM_USED = MISC_OFF + 16;
@@ -124,6 +129,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2], used in the leader only
   uint64_t* mma_done = acc_empty + 2;
+  uint64_t* conv_done = mma_done + 1;   // [2], leader only: accumulator converted to fp32 by the epilogue
+  uint64_t* acc_full2 = conv_done + 2;  // [2]: the outlier MMAs on top of it have completed
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
@@ -150,6 +157,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&acc_empty[b], 2 * EPI_WARPS);
     }
     mbar_init(mma_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&conv_done[b], 2 * EPI_WARPS);
+      mbar_init(&acc_full2[b], 1);
+    }
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -178,14 +189,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   pdl_wait();
   int n_used = 0;
   if (!RAW && !F16 && p.n_used != nullptr) n_used = min(max(*p.n_used, 0), p.out_cap);
-  // Up to 16 outlier columns are added by the epilogue with warp MMAs so the
-  // TMEM accumulators stay double-buffered; more go through tcgen05 fp16 MMAs
-  // into a second accumulator.  The fp16 mode has only fp16 k-blocks (K fp16
-  // columns) and double-buffers their accumulator.
+  // Up to 16 outlier columns are added by the epilogue with warp MMAs.  More
+  // go through tcgen05 fp16 MMAs accumulated on top of the tile's int8 result:
+  // the epilogue first turns the int32 accumulator into fp32 C * SCA / 127 in
+  // place, then the MMA thread adds X[:, O] . CB[:, O]^T into the same TMEM
+  // columns (its k-blocks are issued a few k-blocks into the next tile's
+  // mainloop, by when the conversion is normally done), and the epilogue
+  // scales by SCB / 127.  Both ways keep the two accumulators double-buffered.
+  // The fp16 mode has only fp16 k-blocks (K fp16 columns).
   const bool small_o = !F16 && n_used > 0 && n_used <= SMALL_O && p.XO != nullptr && p.WO != nullptr;
   const int kb_out = F16 ? (K + 63) / 64 : (small_o ? 0 : (n_used + 63) / 64);
-  const int kb_all = kb_int + kb_out;
-  const bool dbl = F16 || kb_out == 0;
+  const bool defer = !F16 && !RAW && kb_out > 0;  // outlier k-blocks issued after the tile's int8 ones
+  const int kb_main = F16 ? kb_out : kb_int;      // k-blocks of a unit's own mainloop
+  const int j_ins = min(4, kb_main - 1);          // a unit's k-block before which the previous
+                                                  // unit's outlier k-blocks are issued
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
@@ -194,7 +211,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t filled = 0, fill_parity = 0;  // leader: per stage, ever filled / parity of the last fill
-      for (int u = pair; u < U.units && !*s_abort; u += npairs) {
+      // one stage: k-block x of map pair (ma, mb) at rows (m0, nb0); false on abort
+      auto load_stage = [&](const CUtensorMap* ma, const CUtensorMap* mb, int x, int m0, int nb0) -> bool {
+        if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.status, p.wait_limit_ns)) return false;
+        uint8_t* sa = smem + stage * STAGE_BYTES;
+        uint8_t* sb = sa + A_BYTES;
+        const uint32_t bar = full0_leader + static_cast<uint32_t>(stage) * 8u;
+        if (leader) {
+          // one arrival that expects the bytes of both CTAs.  The peer's copies
+          // may land first (the transaction count goes negative meanwhile); the
+          // phase cannot complete before this arrival, and the peer cannot
+          // refill the stage before the MMA has consumed it.
+          mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          filled |= 1u << stage;
+          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+        }
+        tma_load_2d_pair(sa, ma, bar, x, m0);
+        tma_load_2d_pair(sb, mb, bar, x, nb0);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
+      // the outlier k-blocks (64 fp16 = 128 bytes deep) of a unit
+      auto load_outliers = [&](int m0, int nb0) -> bool {
+        for (int ko = 0; ko < kb_out; ++ko)
+          if (!load_stage(&tm.XO, &tm.WO, ko * 64, m0, nb0)) return false;
+        return true;
+      };
+      bool ok = true, have_prev = false;
+      int prev_m0 = 0, prev_nb0 = 0;
+      for (int u = pair; ok && u < U.units && !*s_abort; u += npairs) {
         int tile, half;
         U.at(u, tile, half);
         const int m0 = (tile % num_m) * (2 * BM) + static_cast<int>(rank) * BM;
@@ -202,34 +250,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // carries 128 rows; the MMA reads the first 64)
         const int nb0 = (tile / num_m) * BN +
                         (half < 0 ? static_cast<int>(rank) * BNH : half * BNH + static_cast<int>(rank) * (BNH / 2));
-        for (int kb = 0; kb < kb_all; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, s_abort, p.status, p.wait_limit_ns)) break;
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          const uint32_t bar = full0_leader + static_cast<uint32_t>(stage) * 8u;
-          if (leader) {
-            // one arrival that expects the bytes of both CTAs.  The peer's copies
-            // may land first (the transaction count goes negative meanwhile); the
-            // phase cannot complete before this arrival, and the peer cannot
-            // refill the stage before the MMA has consumed it.
-            mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
-            filled |= 1u << stage;
-            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-          }
-          if (kb < kb_int) {
-            tma_load_2d_pair(sa, &tm.A, bar, kb * BK, m0);
-            tma_load_2d_pair(sb, &tm.B, bar, kb * BK, nb0);
-          } else {
-            const int ko = (kb - kb_int) * 64;  // fp16 elements
-            tma_load_2d_pair(sa, &tm.XO, bar, ko, m0);
-            tma_load_2d_pair(sb, &tm.WO, bar, ko, nb0);
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        for (int kb = 0; ok && kb < kb_main; ++kb) {
+          if (defer && have_prev && kb == j_ins) ok = load_outliers(prev_m0, prev_nb0);
+          if (ok) ok = F16 ? load_stage(&tm.XO, &tm.WO, kb * 64, m0, nb0) : load_stage(&tm.A, &tm.B, kb * BK, m0, nb0);
         }
+        prev_m0 = m0;
+        prev_nb0 = nb0;
+        have_prev = true;
       }
+      if (ok && defer && have_prev && !*s_abort) load_outliers(prev_m0, prev_nb0);
       // Never leave while a copy may still be landing in shared memory.  The
       // leader's full barriers count both CTAs' bytes; the peer, which cannot
       // observe them, gives its last copies a bounded grace period.
@@ -249,47 +278,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (leader && lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int it = 0;
-      for (int u = pair; u < U.units && !*s_abort; u += npairs, ++it) {
+      // one stage: 4 MMAs (32 bytes of K each) into accumulator d; false on abort
+      auto mma_stage = [&](uint32_t d, uint32_t idesc, bool f16_block, bool acc0) -> bool {
+        if (!mbar_wait_bounded(&full[stage], phase, s_abort, p.status, p.wait_limit_ns)) return false;
+        tc_fence_after_sync();
+        const uint32_t a_addr = smem_addr(smem + stage * STAGE_BYTES);
+        const uint64_t adesc = smem_desc_k_sw128(a_addr);
+        const uint64_t bdesc = smem_desc_k_sw128(a_addr + A_BYTES);
+        if (f16_block) {
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)  // 16 fp16 = 32 bytes per MMA
+            mma_f16_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, (acc0 || k > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)  // 32 int8 = 32 bytes per MMA
+            mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, (acc0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
+      // the outlier k-blocks of an earlier unit, added on top of its converted
+      // accumulator (fp32 C * SCA / 127 written back by the epilogue)
+      auto outlier_mmas = [&](int b, int nt_b, uint32_t use_b) -> bool {
+        if (!mbar_wait_bounded(&conv_done[b], use_b & 1u, s_abort, p.status, p.wait_limit_ns)) return false;
+        tc_fence_after_sync();
+        const uint32_t idesc_f = idesc_f16_f32(2 * BM, nt_b);
+        for (int ko = 0; ko < kb_out; ++ko)
+          if (!mma_stage(tmem_base + static_cast<uint32_t>(b * BN), idesc_f, true, true)) return false;
+        tc_commit_pair(&acc_full2[b], 0x3);
+        return true;
+      };
+      int it = 0, prev_buf = 0, prev_nt = BN;
+      uint32_t prev_use = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < U.units && !*s_abort; u += npairs, ++it) {
         int tile, half;
         U.at(u, tile, half);
         const int nt = half < 0 ? BN : BNH;
-        const uint32_t idesc_i = idesc_i8_s32(2 * BM, nt);
-        const uint32_t idesc_f = idesc_f16_f32(2 * BM, nt);
-        const int buf = dbl ? (it & 1) : 0;
-        const uint32_t use = dbl ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
+        const uint32_t idesc = F16 ? idesc_f16_f32(2 * BM, nt) : idesc_i8_s32(2 * BM, nt);
+        const int buf = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait_bounded(&acc_empty[buf], (use & 1u) ^ 1u, s_abort, p.status, p.wait_limit_ns)) break;
         tc_fence_after_sync();
-        const uint32_t d_int = tmem_base + static_cast<uint32_t>(buf * BN);
-        const uint32_t d_fp = tmem_base + static_cast<uint32_t>(F16 ? buf * BN : BN);
-        bool ok = true;
-        for (int kb = 0; kb < kb_all; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, s_abort, p.status, p.wait_limit_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          const uint32_t a_addr = smem_addr(smem + stage * STAGE_BYTES);
-          const uint64_t adesc = smem_desc_k_sw128(a_addr);
-          const uint64_t bdesc = smem_desc_k_sw128(a_addr + A_BYTES);
-          if (kb < kb_int) {
-#pragma unroll
-            for (int k = 0; k < BK / 32; ++k)  // 32 int8 = 32 bytes per MMA
-              mma_i8_pair(d_int, adesc + 2 * k, bdesc + 2 * k, idesc_i, (kb > 0 || k > 0) ? 1u : 0u);
-          } else {
-#pragma unroll
-            for (int k = 0; k < BK / 32; ++k)  // 16 fp16 = 32 bytes per MMA
-              mma_f16_pair(d_fp, adesc + 2 * k, bdesc + 2 * k, idesc_f, (kb > kb_int || k > 0) ? 1u : 0u);
-          }
-          tc_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; ok && kb < kb_main; ++kb) {
+          if (defer && it > 0 && kb == j_ins) ok = outlier_mmas(prev_buf, prev_nt, prev_use);
+          if (ok) ok = mma_stage(d, idesc, F16, kb > 0);
         }
         if (!ok) break;
         tc_commit_pair(&acc_full[buf], 0x3);  // both CTAs' accumulator halves are ready
+        prev_buf = buf;
+        prev_nt = nt;
+        prev_use = use;
       }
+      if (ok && defer && it > 0 && !*s_abort) outlier_mmas(prev_buf, prev_nt, prev_use);
       // Wait for every MMA this thread issued before TMEM is released.
       tc_commit_pair(mma_done, 0x1);
       drain_wait(mma_done, 0, p.wait_limit_ns);
@@ -308,6 +354,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int g = lane >> 2, tq = lane & 3;     // fragment row / column pair
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t acc_empty0_leader = map_to_rank(smem_addr(&acc_empty[0]), 0);
+    const uint32_t conv_done0_leader = map_to_rank(smem_addr(&conv_done[0]), 0);
     uint8_t* stg = smem + STG_OFF + ew * 2 * STG_BYTES;
     int stg_i = 0;
     int it = 0;
@@ -319,19 +366,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int nch = half < 0 ? CHUNKS : CHUNKS / 2;
       const int col_off = col_half * nch * 32;  // TMEM column of this warp's first chunk
       const int n0 = (tile / num_m) * BN + (half < 0 ? 0 : half * BNH) + col_off;
-      const int buf = dbl ? (it & 1) : 0;
-      const uint32_t use = dbl ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
+      const int buf = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
       // The chunk loop below is deliberately not unrolled: the epilogue runs
       // beside the TMA and MMA warps, and a compact loop keeps their
       // instructions resident in the instruction cache.  Data a chunk needs
       // besides its accumulators is fetched one chunk ahead (the first chunk's
       // before the accumulator wait).
-      // Row scales of this thread's four rows: row_base + g + 8i.
+      // Row scales of this thread's four rows: row_base + g + 8i (SCA / 127^2,
+      // or SCA / 127 when the outlier MMAs are added on top of the converted
+      // accumulator).
       float sa4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = row_base + g + 8 * i;
-        sa4[i] = (!RAW && !F16 && r < M) ? __ldg(p.SCA + r) * (1.0f / 16129.0f) : 0.f;
+        sa4[i] = (!RAW && !F16 && r < M) ? __ldg(p.SCA + r) * (defer ? (1.0f / 127.0f) : (1.0f / 16129.0f)) : 0.f;
       }
       // Few outliers: the A fragments (X[:, O] rows) of the 16-wide outlier
       // product.  The gathered operands store each group of 16 outlier columns
@@ -385,7 +434,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after_sync();
       const uint32_t t_int = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + col_off);
-      const uint32_t t_fp = tmem_base + lane_off + static_cast<uint32_t>(BN + col_off);
+      if (defer) {
+        // Many outlier columns, phase 1: the int32 accumulator becomes fp32
+        // C * SCA / 127 in place; the MMA thread then adds the outlier product
+        // onto it (fragment element e of row block rb is row rb*16 + g + 8*((e >> 1) & 1)).
+#pragma unroll 1
+        for (int cc = 0; cc < nch; ++cc) {
+          uint32_t c[2][16];
+          tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
+          tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              c[rb][e] = __float_as_uint(static_cast<float>(static_cast<int32_t>(c[rb][e])) * sa4[2 * rb + ((e >> 1) & 1)]);
+          tmem_st_16x256b_x4(t_int + cc * 32, c[0]);
+          tmem_st_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(conv_done0_leader + static_cast<uint32_t>(buf) * 8u);
+        // phase 2: wait until the outlier MMAs of this tile have completed
+        ok = 0;
+        if (lane == 0) ok = mbar_wait_bounded(&acc_full2[buf], use & 1u, s_abort, p.status, p.wait_limit_ns) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        tc_fence_after_sync();
+      }
 #pragma unroll 1
       for (int cc = 0; cc < nch; ++cc) {
         const float sb_c = sb_n, bi_c = bi_n;
@@ -397,17 +473,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         if (cc + 1 < nch) fetch_chunk(cc + 1);
         uint32_t c[2][16];  // int32 accumulators of row blocks 0 / 1
-        if constexpr (!F16) {
+        if (!F16 && !defer) {
           tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
           tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
         }
-        // fp32 accumulators: the outlier product (many-outlier path) or, in the
-        // fp16 mode, the whole product (in the double-buffered columns)
+        // fp32 accumulators: C * SCA / 127 plus the outlier product (many-outlier
+        // path) or, in the fp16 mode, the whole product
         uint32_t f[2][16];
-        if (F16 || (!RAW && kb_out > 0)) {
-          const uint32_t t_f = F16 ? t_int : t_fp;
-          tmem_ld_16x256b_x4(t_f + cc * 32, f[0]);
-          tmem_ld_16x256b_x4(t_f + (16u << 16) + cc * 32, f[1]);
+        if (F16 || defer) {
+          tmem_ld_16x256b_x4(t_int + cc * 32, f[0]);
+          tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, f[1]);
         }
         tmem_wait_ld();
         const int nb = n0 + cc * 32;
@@ -448,7 +523,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             if (small_o) {
               mma_16x8x16_f16(d, af[rb], bf_c[cb][0], bf_c[cb][1]);
-            } else if (kb_out > 0) {
+            } else if (F16 || defer) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) d[e] = __uint_as_float(f[rb][4 * cb + e]);
             }
@@ -456,6 +531,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             for (int hh = 0; hh < 2; ++hh) {
               if constexpr (F16) {
                 halves[rb][cb][hh] = pack_half2(d[2 * hh], d[2 * hh + 1]);
+              } else if (defer) {
+                // (C * SCA / 127 + outlier product) * SCB / 127 + bias
+                halves[rb][cb][hh] = pack_half2(fmaf(d[2 * hh], sb0 * (1.0f / 127.0f), b0),
+                                                fmaf(d[2 * hh + 1], sb1 * (1.0f / 127.0f), b1));
               } else {
                 const float sa = sa4[2 * rb + hh];
                 const float v0 = fmaf(d[2 * hh], sb0 * (1.0f / 127.0f),
@@ -538,13 +617,17 @@ static GemmKernel gemm_kernel(GemmMode mode) {
   }
 }
 
-// Number of CTA pairs that fit on the device at once (cached per mode and device).
+// Number of CTA pairs that fit on the device at once (cached per mode and
+// device; calls may come from several host threads, so the cache is atomic).
 static int max_pairs(GemmMode mode, int num_sms) {
-  static int cache[3][64] = {{0}};
+  static std::atomic<int> cache[3][64];
   int dev = 0;
-  cudaGetDevice(&dev);
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
   const int m = static_cast<int>(mode);
-  if (dev >= 0 && dev < 64 && cache[m][dev] > 0) return cache[m][dev];
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[m][dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1), 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
@@ -562,18 +645,23 @@ static int max_pairs(GemmMode mode, int num_sms) {
     cudaGetLastError();
     n = num_sms / 2;
   }
-  if (dev >= 0 && dev < 64) cache[m][dev] = n;
+  if (dev >= 0 && dev < 64) cache[m][dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, GemmMode mode, int num_sms, cudaStream_t st) {
   if (mode != kGemmFused && mode != kGemmRaw && mode != kGemmF16) return cudaErrorInvalidValue;
-  static bool attr_done[3] = {false, false, false};
+  // the shared-memory opt-in is a per-device property of the kernel: done once
+  // per mode and device (several host threads may get here at once; setting it
+  // twice is harmless)
+  static std::atomic<bool> attr_done[3][64];
   const int m = static_cast<int>(mode);
-  if (!attr_done[m]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !attr_done[m][dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel(mode), cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    attr_done[m] = true;
+    if (dev >= 0 && dev < 64) attr_done[m][dev].store(true, std::memory_order_release);
   }
   const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
   const int pairs_fit = max_pairs(mode, num_sms);

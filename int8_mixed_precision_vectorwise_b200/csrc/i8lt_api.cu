@@ -188,7 +188,9 @@ i8_status run_gemm(const int8_t* A, const int8_t* B, int M, int N, int K, GemmAr
 }
 
 // out [M, Nout] = fp16(Aop [M, Kc] . Bop [Nout, Kc]^T), fp16 operands, fp32 accumulation.
-i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, int Kc, __half* out, cudaStream_t st) {
+// status: optional device word that a pipeline-wait timeout sets to I8_ERR_TIMEOUT.
+i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, int Kc, __half* out, uint32_t* status,
+                       cudaStream_t st) {
   i8lt::GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const uint64_t ld_bytes = static_cast<uint64_t>(Kc) * 2;
@@ -200,6 +202,7 @@ i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, in
   a.N = Nout;
   a.K = Kc;
   a.out = out;
+  a.status = status;
   a.wait_limit_ns = kWaitLimitNs;
   a.tma_store = 0;
   if (Nout % 8 == 0) {
@@ -211,6 +214,29 @@ i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, in
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
   return cuda_status(i8lt::launch_gemm(maps, a, i8lt::kGemmF16, sms, st));
+}
+
+// Few-token GEMM: 128-byte K boxes per pipeline stage (512 bytes of each
+// weight row per stage) and the grid of the stream-K split (one CTA per SM, at
+// most kDecodeMaxGrid, never more CTAs than (tile, stage) work items).
+constexpr int kDecodeBoxes = 4;
+int decode_grid(int N, int K, int sms) {
+  const int total = ((N + 127) / 128) * ((K + 128 * kDecodeBoxes - 1) / (128 * kDecodeBoxes));
+  int grid = sms < i8lt::kDecodeMaxGrid ? sms : i8lt::kDecodeMaxGrid;
+  return grid > total ? total : grid;
+}
+
+// Workspace of the int8 matmul entry point: for few rows, the split-K
+// counters and partial sums of the stream-K kernel; nothing otherwise.
+struct MatmulWs {
+  size_t partials, total;
+};
+MatmulWs matmul_ws_layout(int M, int N, int K) {
+  MatmulWs w{0, 0};
+  if (M > i8lt::kDecodeMaxTokens) return w;
+  w.partials = align256(static_cast<size_t>(decode_counters(N)) * 4);
+  w.total = w.partials + align256(static_cast<size_t>(i8lt::decode_slots(N, K)) * i8lt::kDecodeMaxTokens * N * 8);
+  return w;
 }
 
 }  // namespace
@@ -268,8 +294,8 @@ i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int 
   }
   // status word, counts and bitmap are contiguous: one memset clears them
   if (cudaMemsetAsync(workspace, 0, L.clear_bytes, st) != cudaSuccess) return I8_ERR_CUDA;
-  i8_status s = cuda_status(
-      i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr, st));
+  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr,
+                                                    sms, w.hdr, kWaitLimitNs, st));
   if (s != I8_OK || !outliers) return s;
   return cuda_status(i8lt::launch_outlier_prepare(w.bitmap, K, cap, reinterpret_cast<int32_t*>(w.hdr + 2),
                                                   reinterpret_cast<int32_t*>(w.hdr + 1), w.idx, w.hdr, w.CA, Xh, M,
@@ -308,11 +334,7 @@ i8_status enqueue_gemm(const int8_t* CB, const float* SCB, const i8_half* bias, 
       return I8_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return I8_ERR_CUDA;
-    const int boxes = 4;  // 512 bytes of each weight row per pipeline stage
-    const int total = ((N + 127) / 128) * ((K + 128 * boxes - 1) / (128 * boxes));
-    int grid = sms < i8lt::kDecodeMaxGrid ? sms : i8lt::kDecodeMaxGrid;
-    if (grid > total) grid = total;
-    return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, grid, boxes, st));
+    return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms), kDecodeBoxes, true, st));
   }
   GemmArgs a{};
   a.M = M;
@@ -339,6 +361,39 @@ i8_status enqueue_matmul_dequant(const int8_t* CB, const float* SCB, const i8_ha
   return enqueue_gemm(CB, SCB, bias, M, N, K, threshold, out, w, w.counters, w.WO, cap, L, st);
 }
 
+// Small problems run the whole forward as one kernel (k_linear_small): few
+// tokens, a row of X that fits the kernel's shared-memory code tile, a weight
+// of at most 8 MiB spread over at most one CTA per SM, and an outlier capacity
+// the kernel's list holds.  Everything else runs the two-stage path.
+constexpr size_t kSmallMaxWeightBytes = size_t(8) << 20;
+bool use_small(int M, int N, int K, int cap) {
+  if (M > i8lt::kDecodeMaxTokens || K > i8lt::kSmallMaxK || cap > i8lt::kSmallListCap) return false;
+  if (static_cast<size_t>(N) * K > kSmallMaxWeightBytes) return false;
+  const int sms = num_sms();
+  return sms > 0 && (N + 127) / 128 <= sms;
+}
+
+// One weight's forward with the prepared quantities kept on chip; the kernel
+// writes the status word and outlier counts of the workspace header.
+i8_status enqueue_small(const i8_half* X, const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N,
+                        int K, float threshold, i8_half* out, void* workspace, int cap, cudaStream_t st) {
+  CUtensorMap tmW;
+  if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, CB, K, N, K, 128, 128)) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_linear_small(tmW, reinterpret_cast<const __half*>(X), M, N, K, threshold, cap, SCB,
+                                               reinterpret_cast<const __half*>(bias), reinterpret_cast<__half*>(out),
+                                               static_cast<uint32_t*>(workspace), kWaitLimitNs, true, st));
+}
+
+// The forward of one weight on a workspace laid out by ws_layout.
+i8_status enqueue_forward(const i8_half* X, const int8_t* CB, const float* SCB, const i8_half* bias, int M, int N,
+                          int K, float threshold, i8_half* out, void* workspace, int cap, const WsLayout& L,
+                          cudaStream_t st) {
+  if (use_small(M, N, K, cap)) return enqueue_small(X, CB, SCB, bias, M, N, K, threshold, out, workspace, cap, st);
+  i8_status s = enqueue_prepare(X, CB, M, N, K, threshold, workspace, cap, L, st);
+  if (s != I8_OK) return s;
+  return enqueue_matmul_dequant(CB, SCB, bias, M, N, K, threshold, out, workspace, cap, L, st);
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- allocation-free forward
@@ -350,19 +405,50 @@ static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 namespace {
 
+// Unique id of the calling thread's current CUDA context (driver ids are never
+// reused within a process), or 0 if the driver cannot say.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 // Device address of g_static_scratch on the current device.  In host code the
 // array's name only stands in for the symbol, so the address is looked up with
-// cudaGetSymbolAddress, once per device, while that device is current.
+// cudaGetSymbolAddress while that device is current: once per device and
+// context.  If the device's context is torn down and created again (the module
+// is then loaded again and the array may move), the new context id triggers a
+// fresh lookup.
 i8_status static_scratch(void** out) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
+  static unsigned long long ctx_of[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return I8_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return I8_ERR_CUDA;
     addr[dev] = p;
+    ctx_of[dev] = current_context_id();  // the lookup has made the device's context current
   }
   *out = addr[dev];
   return I8_OK;
@@ -400,8 +486,8 @@ i8_status i8_quantize_rowwise(const i8_half* X, int M, int K, float threshold, i
   }
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
-  i8_status s = cuda_status(
-      i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, threshold > 0.f ? bitmap : nullptr, st));
+  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, threshold > 0.f ? bitmap : nullptr,
+                                                    sms, nullptr, kWaitLimitNs, st));
   if (s != I8_OK || threshold == 0.f) return s;
   return cuda_status(i8lt::launch_zero_outlier_cols(bitmap, M, K, CA, sms, st));
 }
@@ -431,6 +517,76 @@ i8_status i8_int8_linear_matmul(const int8_t* A, const int8_t* B, int M, int N, 
   a.C = C;
   a.wait_limit_ns = kWaitLimitNs;
   return run_gemm(A, B, M, N, K, a, true, nullptr, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t i8_int8_linear_matmul_workspace_size(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return matmul_ws_layout(M, N, K).total;
+}
+
+i8_status i8_int8_linear_matmul_ws(const int8_t* A, const int8_t* B, int M, int N, int K, int32_t* C, void* workspace,
+                                   size_t workspace_bytes, uint32_t* status, i8_stream_t stream) {
+  i8_status s = check_gemm_operands(A, B, M, N, K);
+  if (s != I8_OK) return s;
+  if (!C) return I8_ERR_INVALID_ARG;
+  if (!aligned16(C)) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (status && (reinterpret_cast<uintptr_t>(status) & 3u) != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  const MatmulWs w = matmul_ws_layout(M, N, K);
+  if (w.total > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+                      workspace_bytes < w.total))
+    return I8_ERR_WORKSPACE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (status && cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return I8_ERR_CUDA;
+  if (M > i8lt::kDecodeMaxTokens) {
+    GemmArgs a{};
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.C = C;
+    a.status = status;
+    a.wait_limit_ns = kWaitLimitNs;
+    return run_gemm(A, B, M, N, K, a, true, nullptr, nullptr, 0, st);
+  }
+  // Few rows: the forward's stream-K kernel, storing its int32 sums.  Its
+  // split-K counters must start at zero.
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, w.partials, st) != cudaSuccess) return I8_ERR_CUDA;
+  i8lt::DecodeArgs d{};
+  d.M = M;
+  d.N = N;
+  d.K = K;
+  d.C = C;
+  d.partials = reinterpret_cast<int32_t*>(ws + w.partials);
+  d.slots = i8lt::decode_slots(N, K);
+  d.counters = reinterpret_cast<int32_t*>(ws);
+  d.status = status;
+  d.wait_limit_ns = kWaitLimitNs;
+  CUtensorMap tmW, tmC;
+  if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, 128, 128) ||
+      !encode_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, 128, i8lt::kDecodeMaxTokens))
+    return I8_ERR_CUDA;
+  // no programmatic overlap: B may be written by the work queued just before
+  return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms), kDecodeBoxes, false, st));
+}
+
+i8_status i8_linear8bit_workspace_layout(int M, int N, int K, int max_outlier_cols, i8_workspace_layout* layout) {
+  if (!layout) return I8_ERR_INVALID_ARG;
+  if (max_outlier_cols > kMaxOutlierCap) return I8_ERR_UNSUPPORTED_SHAPE;
+  WsLayout L;
+  if (N <= 0 || !ws_layout(M, N, K, max_outlier_cols, &L)) return I8_ERR_INVALID_ARG;
+  layout->header = L.hdr;
+  layout->bitmap = L.bitmap;
+  layout->idx = L.idx;
+  layout->sca = L.sca;
+  layout->ca = L.ca;
+  layout->x_o = L.xo;
+  layout->w_o = L.wo;
+  layout->total = L.total;
+  layout->ld_o = L.ld_o;
+  layout->few_tokens = L.decode ? 1 : 0;
+  return I8_OK;
 }
 
 i8_status i8_int8_mm_dequant(const int32_t* C, const float* SCA, const float* SCB, const i8_half* bias, int M,
@@ -467,14 +623,34 @@ i8_status i8_dequant_transposed(const int8_t* CB, const float* SCB, int N, int K
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
-i8_status i8_linear8bit_backward_input(const i8_half* dY, const i8_half* Wt, int M, int N, int K, i8_half* dX,
-                                       i8_stream_t stream) {
+i8_status i8_gather_column_blocks(const i8_half* G, int P, int M, int Np, i8_half* out, i8_stream_t stream) {
+  if (!G || !out) return I8_ERR_INVALID_ARG;
+  if (P <= 0 || M <= 0 || Np <= 0) return I8_ERR_INVALID_ARG;
+  if (static_cast<long long>(P) * Np > (1LL << 31) - 1) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(G) || !aligned16(out)) return I8_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_gather_column_blocks(reinterpret_cast<const __half*>(G), P, M, Np,
+                                                       reinterpret_cast<__half*>(out), sms,
+                                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_linear8bit_backward_input_status(const i8_half* dY, const i8_half* Wt, int M, int N, int K,
+                                              i8_half* dX, uint32_t* status, i8_stream_t stream) {
   if (!dY || !Wt || !dX) return I8_ERR_INVALID_ARG;
   if (M <= 0 || N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
   if (N % 8 != 0) return I8_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(dY) || !aligned16(Wt) || !aligned16(dX)) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (status && (reinterpret_cast<uintptr_t>(status) & 3u) != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (status && cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return I8_ERR_CUDA;
   return run_gemm_f16(reinterpret_cast<const __half*>(dY), reinterpret_cast<const __half*>(Wt), M, K, N,
-                      reinterpret_cast<__half*>(dX), reinterpret_cast<cudaStream_t>(stream));
+                      reinterpret_cast<__half*>(dX), status, st);
+}
+
+i8_status i8_linear8bit_backward_input(const i8_half* dY, const i8_half* Wt, int M, int N, int K, i8_half* dX,
+                                       i8_stream_t stream) {
+  return i8_linear8bit_backward_input_status(dY, Wt, M, N, K, dX, nullptr, stream);
 }
 
 size_t i8_linear8bit_workspace_size(int M, int N, int K, int max_outlier_cols) {
@@ -513,10 +689,8 @@ i8_status i8_linear8bit_forward(const i8_half* X, const int8_t* CB, const float*
   i8_status s = check_forward(X, CB, SCB, bias, M, N, K, threshold, out, true, workspace, workspace_bytes,
                               max_outlier_cols, &L);
   if (s != I8_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  s = enqueue_prepare(X, CB, M, N, K, threshold, workspace, max_outlier_cols, L, st);
-  if (s != I8_OK) return s;
-  return enqueue_matmul_dequant(CB, SCB, bias, M, N, K, threshold, out, workspace, max_outlier_cols, L, st);
+  return enqueue_forward(X, CB, SCB, bias, M, N, K, threshold, out, workspace, max_outlier_cols, L,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t i8_linear8bit_multi_workspace_size(int M, int K, int G, const int* N, int max_outlier_cols) {
@@ -542,19 +716,37 @@ i8_status i8_linear8bit_forward_multi(const i8_half* X, int M, int K, int G, con
   if (!ws_layout_multi(M, K, G, N, cap, &L)) return I8_ERR_INVALID_ARG;
   if (workspace_bytes < L.total) return I8_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // X is quantised and its outlier columns found once; the first weight's
-  // outlier rows are gathered in the same launch
-  i8_status s = enqueue_prepare(X, CB[0], M, N[0], K, threshold, workspace, cap, L, st);
-  if (s != I8_OK) return s;
+  // Every weight runs as its own forward would: small ones as the one-launch
+  // kernel, the rest on X quantised (and its outlier columns found) once, the
+  // first of them with its outlier rows gathered in the same launch.
+  int first_big = -1;
+  for (int g = 0; g < G && first_big < 0; ++g)
+    if (!use_small(M, N[g], K, cap)) first_big = g;
+  i8_status s = I8_OK;
+  if (first_big >= 0) {
+    s = enqueue_prepare(X, CB[first_big], M, N[first_big], K, threshold, workspace, cap, L, st);
+    if (s != I8_OK) return s;
+  }
   const WsPtrs w = ws_ptrs(workspace, L);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool gather_w = !L.decode && threshold > 0.f && cap > 0;
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
   for (int g = 0; g < G; ++g) {
+    if (use_small(M, N[g], K, cap)) {
+      // the status word is reset by the first operation of the call only
+      const bool reset = first_big < 0 && g == 0;
+      CUtensorMap tmW;
+      if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, CB[g], K, N[g], K, 128, 128)) return I8_ERR_CUDA;
+      s = cuda_status(i8lt::launch_linear_small(tmW, reinterpret_cast<const __half*>(X), M, N[g], K, threshold, cap,
+                                                SCB[g], reinterpret_cast<const __half*>(bias ? bias[g] : nullptr),
+                                                reinterpret_cast<__half*>(out[g]), w.hdr, kWaitLimitNs, reset, st));
+      if (s != I8_OK) return s;
+      continue;
+    }
     __half* WO = reinterpret_cast<__half*>(ws + wo_offset(L, N, g));
     int32_t* counters = reinterpret_cast<int32_t*>(ws + counters_offset(L, N, g));
-    if (g > 0 && gather_w) {
+    if (g != first_big && gather_w) {
       // this weight's outlier rows only: the list is rebuilt from the bitmap, X is not touched
       s = cuda_status(i8lt::launch_outlier_prepare(w.bitmap, K, cap, nullptr, nullptr, nullptr, nullptr, nullptr,
                                                    nullptr, 0, nullptr, CB[g], N[g], WO, L.ld_o, sms, st));
@@ -600,11 +792,10 @@ i8_status i8_linear8bit_forward_static(const i8_half* X, const int8_t* CB, const
   s = static_scratch(&ws);
   if (s != I8_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // the prepare stage clears the status word, counts and bitmap; every other
-  // byte it reads back is written earlier in the same call
-  s = enqueue_prepare(X, CB, M, N, K, threshold, ws, max_outlier_cols, L, st);
-  if (s != I8_OK) return s;
-  s = enqueue_matmul_dequant(CB, SCB, bias, M, N, K, threshold, out, ws, max_outlier_cols, L, st);
+  // the same kernels as i8_linear8bit_forward: the first of them clears (or
+  // writes) the status word and counts; every other byte read back is written
+  // earlier in the same call
+  s = enqueue_forward(X, CB, SCB, bias, M, N, K, threshold, out, ws, max_outlier_cols, L, st);
   if (s != I8_OK || status_out == nullptr) return s;
   return cuda_status(cudaMemcpyAsync(status_out, ws, 3 * sizeof(uint32_t), cudaMemcpyDeviceToDevice, st));
 }

@@ -9,9 +9,10 @@
 
 namespace i8lt {
 
-// bitmap: zeroed outlier bitmap to OR into (required when tau > 0).
+// bitmap: zeroed outlier bitmap to OR into (required when tau > 0).  status
+// (nullable): device word that a pipeline-wait timeout of the ring kernel sets.
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
-                              cudaStream_t st);
+                              int num_sms, uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 cudaError_t launch_zero_outlier_cols(const uint32_t* bitmap, int M, int K, int8_t* CA, int num_sms,
                                      cudaStream_t st);
 cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32_t* total_out, int32_t* used_out,
@@ -24,6 +25,9 @@ cudaError_t launch_dequant(const int8_t* CB, const float* SCB, int N, int K, __h
                            cudaStream_t st);
 // Wt [K, N] = the transpose of launch_dequant's W (K % 16 == 0, N % 8 == 0).
 cudaError_t launch_dequant_t(const int8_t* CB, const float* SCB, int N, int K, __half* Wt, cudaStream_t st);
+// out [M, P*Np] from P rank-major column blocks G [P, M, Np].
+cudaError_t launch_gather_column_blocks(const __half* G, int P, int M, int Np, __half* out, int num_sms,
+                                        cudaStream_t st);
 
 // Tensor-core GEMM (tcgen05, TMA-fed, TMEM accumulators).
 struct GemmArgs {
@@ -92,6 +96,8 @@ struct DecodeArgs {
   int32_t* counters;         // [ceil(N/128) * 4], zero on entry
   uint32_t* status;
   uint64_t wait_limit_ns;
+  int32_t* C;                // raw mode when non-null: C[t, n] = sum_k CA[t, k] * CB[n, k] as int32 [M, N]
+                             // (no scales, bias or outlier term are read; out is not written)
 };
 
 // Partial-sum slots the decode GEMM needs for these sizes (grid <= kDecodeMaxGrid).
@@ -104,8 +110,11 @@ inline int decode_slots(int N, int K) {
 
 // tmW: CB [N, K] int8, box 128 rows x 128 B; tmC: CA [M, K] int8, box 16 rows x 128 B.
 // boxes_per_stage: 128-byte K boxes per pipeline stage (1, 2 or 4).
+// pdl: launch as a programmatic dependent of the kernel before it on the
+// stream (the weights are then requested before that kernel has finished, so
+// it must not write CB).
 cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
-                               int boxes_per_stage, cudaStream_t st);
+                               int boxes_per_stage, bool pdl, cudaStream_t st);
 
 // Few-token preparation on one cluster of kDecodePrepCluster CTAs (M <= 16):
 // codes, SCA, outlier list, X_O (zero padded to a multiple of 16 columns), the
@@ -115,6 +124,19 @@ constexpr int kDecodePrepCluster = 8;
 cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA,
                                int32_t* idx, __half* XO, int ld_o, uint32_t* hdr, int32_t* counters, int n_counters,
                                cudaStream_t st);
+
+// The whole forward of a small problem in one launch (M <= 16 tokens,
+// K <= kSmallMaxK, at most kSmallListCap outlier columns): one CTA per 128
+// weight rows quantises X itself and runs its tile on the tensor cores.
+// tmW: CB [N, K] int8, box 128 rows x 128 B.  hdr: status word, used and total
+// outlier counts (the counts are written by the kernel; the status word is
+// set when reset_status, else only raised to an error).  bias may be null.
+constexpr int kSmallMaxK = 4096;
+constexpr int kSmallListCap = 512;
+size_t linear_small_smem(int K);
+cudaError_t launch_linear_small(const CUtensorMap& tmW, const __half* X, int M, int N, int K, float tau, int cap,
+                                const float* SCB, const __half* bias, __half* out, uint32_t* hdr, uint64_t limit_ns,
+                                bool reset_status, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 

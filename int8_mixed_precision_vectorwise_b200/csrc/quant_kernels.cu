@@ -11,6 +11,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -166,6 +167,104 @@ __global__ void __launch_bounds__(256, (VPT > 8 ? 1 : 5)) k_quant_rows(const __h
   }
 }
 
+// Persistent ring quantiser for rows of 2 KB .. 32 KB (1024 <= K <= 16384).
+// Each CTA (one per SM) owns a contiguous range of rows.  Lane 0 of warp 0
+// streams whole rows of X into a ring of shared-memory slots with 1-D bulk
+// copies, so up to `slots` rows (~200 KB) per SM are in flight while rows are
+// being quantised; a slot is refilled as soon as the row in it is done.  The
+// other 8 warps quantise one row at a time together, from shared memory:
+// absmax over the row (elements at or above the threshold left out and marked
+// in the CTA's outlier bitmap), one fp32 division, codes written with 8-byte
+// coalesced stores.  Every wait is bounded; a timeout sets *status (when
+// given) and all warps leave together (the per-row barrier also ORs the
+// warps' failures), the producer first waiting, bounded, for its copies.
+constexpr int kRingConsumers = 256;  // threads that quantise a row together
+constexpr int kRingThreads = 32 + kRingConsumers;
+constexpr int kRingMaxSlots = 32;
+constexpr int kRingSlotBudget = 200 * 1024;
+
+__global__ void __launch_bounds__(kRingThreads, 1)
+    k_quant_rows_ring(const __half* __restrict__ X, int M, int K, float tau, int8_t* __restrict__ CA,
+                      float* __restrict__ SCA, uint32_t* __restrict__ bitmap, int rows_per_cta, int slots,
+                      uint32_t* status, uint64_t limit_ns) {
+  extern __shared__ __align__(128) uint8_t rsm[];
+  const int row_bytes = 2 * K;
+  uint8_t* ring = rsm;
+  uint64_t* full = reinterpret_cast<uint64_t*>(rsm + static_cast<size_t>(slots) * row_bytes);
+  uint64_t* empty = full + slots;
+  float* red = reinterpret_cast<float*>(empty + slots);  // [2][8]: row parity x consumer warp
+  volatile int* s_abort = reinterpret_cast<volatile int*>(red + 16);
+  uint32_t* sbm = reinterpret_cast<uint32_t*>(red + 20);
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = blockIdx.x * rows_per_cta;
+  const int n = max(0, min(rows_per_cta, M - r0));
+  const int nvec = K >> 3, nwords = (K + 31) >> 5;
+  const bool use_tau = tau > 0.f;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < slots; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kRingConsumers / 32);
+    }
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (use_tau) sbm_clear(sbm, nwords);
+  __syncthreads();
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      uint32_t filled = 0, fill_parity = 0;
+      for (int j = 0; j < n; ++j) {
+        const int s = j % slots;
+        const uint32_t use = static_cast<uint32_t>(j / slots);
+        if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1u, s_abort, status, limit_ns)) break;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(row_bytes));
+        filled |= 1u << s;
+        fill_parity = (fill_parity & ~(1u << s)) | ((use & 1u) << s);
+        bulk_load(ring + static_cast<size_t>(s) * row_bytes, X + static_cast<size_t>(r0 + j) * K,
+                  static_cast<uint32_t>(row_bytes), &full[s]);
+      }
+      if (*s_abort) {  // never leave while a copy may still be landing in shared memory
+        int never = 0;
+        for (int s = 0; s < slots; ++s)
+          if (filled & (1u << s)) mbar_wait_bounded(&full[s], (fill_parity >> s) & 1u, &never, nullptr, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int t = threadIdx.x - 32, cw = warp - 1;
+    for (int j = 0; j < n; ++j) {
+      const int s = j % slots;
+      const uint32_t parity = static_cast<uint32_t>(j / slots) & 1u;
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded(&full[s], parity, s_abort, status, limit_ns) ? 1 : 0;
+      ok = __shfl_sync(kFull, ok, 0);
+      const uint4* v = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(s) * row_bytes);
+      float amax = 0.f;
+      if (ok)
+        for (int vi = t; vi < nvec; vi += kRingConsumers) fold8(v[vi], vi, tau, use_tau, amax, sbm);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+      if (lane == 0) red[(j & 1) * 8 + cw] = amax;
+      if (named_bar_any(1, kRingConsumers, !ok)) break;  // every consumer warp leaves at the same row
+      amax = red[(j & 1) * 8];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[(j & 1) * 8 + w]);
+      const float r = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
+      const int row = r0 + j;
+      if (t == 0) SCA[row] = amax;
+      uint2* cr = reinterpret_cast<uint2*>(CA + static_cast<size_t>(row) * K);
+      for (int vi = t; vi < nvec; vi += kRingConsumers) cr[vi] = quant8(v[vi], r);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the slot
+    }
+  }
+  __syncthreads();
+  if (use_tau) sbm_flush(sbm, nwords, bitmap);
+}
+
 // Rows too long to cache in registers: one block per row, X read twice (the
 // second read is served by L2).
 __global__ void __launch_bounds__(256) k_quant_rows_stream(const __half* __restrict__ X, int M, int K,
@@ -229,11 +328,16 @@ __device__ __forceinline__ int outlier_slot(int pos) {
 }
 
 // Outlier preparation for the fused forward.  Every block rebuilds the sorted
-// column list from the bitmap in shared memory (a block-wide scan of popcounts),
-// then the grid's threads walk rows, one row each: X rows (zero CA[:, O],
-// gather X[:, O]) and CB rows (gather fp16(CB[:, O])).  Gathered rows are zero-padded to a multiple
-// of 64 columns (one 128-byte fp16 tile).  Block 0 publishes the list, the
-// counts and the overflow status.
+// column list from the bitmap in shared memory (a block-wide scan of
+// popcounts); then the grid's threads take work items (row, group of 16 list
+// positions) over the X rows (gather X[:, O] into X_O, zero CA[:, O]) and the
+// CB rows (gather fp16(CB[:, O]) into W_O).  An item issues its 16 gathers at
+// once and writes the group as two 16-byte stores, so the scattered reads of
+// every (row, column) pair are in flight together across the grid.  Up to 16
+// used columns the operands are written as one zero-padded group of 16 (the
+// GEMM's epilogue reads exactly that); past 16, zero padded to a multiple of
+// 64 (one 128-byte fp16 tile of the tensor-core path).  Block 0 publishes the
+// list, the counts and the overflow status.
 __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restrict__ bitmap, int K, int cap,
                                                          int32_t* __restrict__ total_out,
                                                          int32_t* __restrict__ used_out,
@@ -295,41 +399,45 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
     }
   }
   if (used == 0) return;
-  const int n_pad = (used + 63) & ~63;
+  const int groups = used <= 16 ? 1 : ((used + 63) & ~63) >> 4;  // 16-position groups written
   const int rows_x = (XO != nullptr || CA != nullptr) ? M : 0;
   const int rows_w = WO != nullptr ? N : 0;
-  // One thread per row: its `used` gathers are independent loads issued
-  // together, then the gathered row (zero padded) leaves as 16-byte stores.
-  for (int r = blockIdx.x * 256 + threadIdx.x; r < rows_x + rows_w; r += gridDim.x * 256) {
+  const long long items = static_cast<long long>(rows_x + rows_w) * groups;
+  for (long long it = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; it < items;
+       it += static_cast<long long>(gridDim.x) * 256) {
+    const int r = static_cast<int>(it / groups);
+    const int p0 = static_cast<int>(it - static_cast<long long>(r) * groups) * 16;  // first stored position
     const bool is_x = r < rows_x;
     const int row = is_x ? r : r - rows_x;
     const size_t base = static_cast<size_t>(row) * K;
     __half* dst = is_x ? (XO != nullptr ? XO + static_cast<size_t>(row) * ld_o : nullptr)
                        : WO + static_cast<size_t>(row) * ld_o;
-    for (int c0 = 0; c0 < n_pad; c0 += 8) {
-      uint32_t h[4] = {0u, 0u, 0u, 0u};
-      if ((c0 & ~15) < used) {  // the 16-column group holds list entries
-        unsigned short v[8];
+    uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (p0 < used) {  // the group holds list entries; the rest of the padding stays 0
+      unsigned short v[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          // stored position c0 + q holds list entry outlier_slot(c0 + q)
-          const int c = outlier_slot(c0 + q);
-          v[q] = 0;
-          if (c < used) {
-            const int j = idx_s[c];
-            v[q] = is_x ? __half_as_ushort(X[base + j])
-                        : __half_as_ushort(__int2half_rn(static_cast<int>(CB[base + j])));
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) h[q] = static_cast<uint32_t>(v[2 * q]) | (static_cast<uint32_t>(v[2 * q + 1]) << 16);
-        if (is_x && CA != nullptr) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (c0 + q < used) CA[base + idx_s[c0 + q]] = 0;  // every listed column, in list order
+      for (int q = 0; q < 16; ++q) {
+        // stored position p0 + q holds list entry outlier_slot(p0 + q)
+        const int c = outlier_slot(p0 + q);
+        v[q] = 0;
+        if (c < used) {
+          const int j = idx_s[c];
+          v[q] = is_x ? __half_as_ushort(X[base + j])
+                      : __half_as_ushort(__int2half_rn(static_cast<int>(CB[base + j])));
         }
       }
-      if (dst != nullptr) *reinterpret_cast<uint4*>(dst + c0) = make_uint4(h[0], h[1], h[2], h[3]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) h[q] = static_cast<uint32_t>(v[2 * q]) | (static_cast<uint32_t>(v[2 * q + 1]) << 16);
+      if (is_x && CA != nullptr) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (p0 + q < used) CA[base + idx_s[p0 + q]] = 0;  // the group's columns, in list order
+      }
+    }
+    if (dst != nullptr) {
+      uint4* d = reinterpret_cast<uint4*>(dst + p0);
+      d[0] = make_uint4(h[0], h[1], h[2], h[3]);
+      d[1] = make_uint4(h[4], h[5], h[6], h[7]);
     }
   }
 }
@@ -434,11 +542,65 @@ __global__ void __launch_bounds__(256) k_dequant_t(const int8_t* __restrict__ CB
   }
 }
 
+// Column blocks gathered from P ranks, G [P, M, Np] (rank-major, as an
+// all-gather of each rank's [M, Np] output leaves them), laid out as the
+// output of the whole layer: out[m, p * Np + j] = G[p, m, j].  16 bytes per
+// thread when Np % 8 == 0, else one element.
+__global__ void __launch_bounds__(256) k_gather_column_blocks(const __half* __restrict__ G, int P, int M, int Np,
+                                                              __half* __restrict__ out) {
+  const bool vec = (Np & 7) == 0;
+  const int per_row = vec ? Np >> 3 : Np;  // units per (rank, row)
+  const size_t units = static_cast<size_t>(P) * M * per_row;
+  const size_t N = static_cast<size_t>(P) * Np;
+  for (size_t u = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; u < units;
+       u += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t pm = u / per_row;
+    const int j = static_cast<int>(u - pm * per_row);
+    const int p = static_cast<int>(pm / M), m = static_cast<int>(pm - static_cast<size_t>(p) * M);
+    if (vec) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(G + pm * Np) + j);
+      *reinterpret_cast<uint4*>(out + m * N + static_cast<size_t>(p) * Np + 8 * j) = v;
+    } else {
+      out[m * N + static_cast<size_t>(p) * Np + j] = G[pm * Np + j];
+    }
+  }
+}
+
+cudaError_t launch_gather_column_blocks(const __half* G, int P, int M, int Np, __half* out, int num_sms,
+                                        cudaStream_t st) {
+  const size_t units = static_cast<size_t>(P) * M * ((Np & 7) == 0 ? Np / 8 : Np);
+  const int blocks = static_cast<int>(std::min<size_t>((units + 255) / 256, static_cast<size_t>(num_sms) * 8));
+  k_gather_column_blocks<<<std::max(blocks, 1), 256, 0, st>>>(G, P, M, Np, out);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
-                              cudaStream_t st) {
+                              int num_sms, uint32_t* status, uint64_t limit_ns, cudaStream_t st) {
   const size_t smem = tau > 0.f ? static_cast<size_t>((K + 31) / 32) * 4 : 0;
   const int nvec = K / 8;
+  if (K >= 1024 && K <= 16384 && num_sms > 0) {
+    // rows of 2 KB .. 32 KB: the persistent ring kernel, one CTA per SM
+    const int row_bytes = 2 * K;
+    const int slots = std::min(kRingMaxSlots, kRingSlotBudget / row_bytes);
+    const size_t ring_smem = static_cast<size_t>(slots) * row_bytes + static_cast<size_t>(slots) * 16 + 20 * 4 +
+                             static_cast<size_t>((K + 31) / 32) * 4;
+    static std::atomic<bool> attr_done[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
+      cudaError_t e = cudaFuncSetAttribute(k_quant_rows_ring, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kRingSlotBudget + 8 * 1024);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
+    }
+    int grid = std::min(M, num_sms);
+    const int rows_per_cta = (M + grid - 1) / grid;
+    grid = (M + rows_per_cta - 1) / rows_per_cta;
+    k_quant_rows_ring<<<grid, kRingThreads, ring_smem, st>>>(X, M, K, tau, CA, SCA, bitmap, rows_per_cta, slots,
+                                                              status, limit_ns);
+    return cudaGetLastError();
+  }
   // One row per group of threads with the row in registers (one pass over X),
   // grids of many small blocks so that enough rows are in flight per SM; rows
   // beyond 32768 columns stream twice.
@@ -469,8 +631,11 @@ cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32
                                    int32_t* idx_out, uint32_t* status, int8_t* CA, const __half* X, int M,
                                    __half* XO, const int8_t* CB, int N, __half* WO, int ld_o, int num_sms,
                                    cudaStream_t st) {
+  // work items: (row, 16-position group); a grid of up to 8 blocks per SM
   const int rows = ((XO || CA) ? M : 0) + (WO ? N : 0);
-  const int blocks = max(1, min((rows + 255) / 256, num_sms * 4));
+  const int groups = cap <= 16 ? 1 : ((cap + 63) / 64) * 4;
+  const long long items = static_cast<long long>(rows) * groups;
+  const int blocks = static_cast<int>(std::max<long long>(1, std::min<long long>((items + 255) / 256, num_sms * 8LL)));
   const size_t smem = static_cast<size_t>(max(cap, 1)) * sizeof(int32_t);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks, 1, 1);
