@@ -171,3 +171,60 @@ def test_binding_shape_and_device_checks():
         b._arg(t, torch.float16, "t", (3, 4), torch.device("cpu"))       # inputs must live on the GPU
     with pytest.raises(TypeError, match="float16"):
         b._arg(t.float(), torch.float16, "t", (3, 4), torch.device("cpu"))
+
+
+def test_matmul_ws_size_and_rejects(lib):
+    lib.i8_int8_linear_matmul_workspace_size.restype = ctypes.c_size_t
+    sz = lib.i8_int8_linear_matmul_workspace_size
+    assert sz(17, 4096, 4096) == 0                       # many rows: the tensor-core GEMM needs none
+    assert sz(0, 4096, 4096) == 0 and sz(4, -1, 16) == 0
+    n16 = sz(16, 28672, 8192)
+    # split-K counters (4 per 128-row tile) and the int32 + fp32 partial sums of every slot
+    assert n16 >= (28672 // 128) * 4 * 4 + 16 * 28672 * 8
+    assert sz(1, 28672, 8192) == n16                      # sized for 16 token columns whatever M is
+    f = lib.i8_int8_linear_matmul_ws
+    S = ctypes.c_size_t
+    assert f(None, FAKE, 4, 4, 16, FAKE, FAKE, S(n16), None, None) == 1
+    assert f(FAKE, FAKE, 4, 4, 40, FAKE, FAKE, S(n16), None, None) == 2    # K % 16
+    assert f(FAKE, FAKE, 4, 4, 16, None, FAKE, S(n16), None, None) == 1    # C
+    need = sz(4, 4, 16)
+    assert need > 0
+    assert f(FAKE, FAKE, 4, 4, 16, FAKE, None, S(need), None, None) == 3   # few rows need a workspace
+    assert f(FAKE, FAKE, 4, 4, 16, FAKE, FAKE, S(need - 1), None, None) == 3
+    assert f(FAKE, FAKE, 4, 4, 16, FAKE, ctypes.c_void_p(0x1010), S(need), None, None) == 3
+    assert f(FAKE, FAKE, 4, 4, 16, FAKE, FAKE, S(need), ctypes.c_void_p(0x1002), None) == 2  # status alignment
+
+
+def test_backward_status_rejects(lib):
+    g = lib.i8_linear8bit_backward_input_status
+    assert g(None, FAKE, 4, 8, 16, FAKE, FAKE, None) == 1
+    assert g(FAKE, FAKE, 4, 12, 16, FAKE, FAKE, None) == 2
+    assert g(FAKE, FAKE, 4, 8, 16, FAKE, ctypes.c_void_p(0x1001), None) == 2
+
+
+def test_workspace_layout_matches_size():
+    from int8_mixed_precision_vectorwise_b200 import _binding as b
+    lib = b.lib()
+    lib.i8_linear8bit_workspace_size.restype = ctypes.c_size_t
+    for M, N, K, cap in [(1, 28672, 8192, 256), (16, 1024, 1024, 8), (17, 4096, 4096, 256), (300, 520, 1040, 64),
+                         (4096, 11008, 4096, 0)]:
+        L = b.i8_linear8bit_workspace_layout(M, N, K, cap)
+        assert L["total"] == lib.i8_linear8bit_workspace_size(M, N, K, cap)
+        assert L["few_tokens"] == int(M <= 16)
+        assert L["ld_o"] == (0 if cap == 0 else -(-cap // 64) * 64)
+        # regions in order, 256-byte aligned, large enough for what they hold
+        order = ["header", "bitmap", "idx", "sca", "ca", "x_o", "w_o"]
+        offs = [L[k] for k in order]
+        assert all(o % 256 == 0 for o in offs)
+        assert offs == sorted(offs)
+        assert L["bitmap"] - L["header"] >= 12
+        assert L["sca"] - L["idx"] >= 4 * max(cap, 1)
+        assert L["ca"] - L["sca"] >= 4 * M
+        assert L["x_o"] - L["ca"] >= M * K
+        assert L["w_o"] - L["x_o"] >= 2 * M * L["ld_o"]
+        if M > 16:
+            assert L["total"] - L["w_o"] >= 2 * N * L["ld_o"]
+    with pytest.raises(b.I8Error):
+        b.i8_linear8bit_workspace_layout(0, 4, 16, 8)
+    with pytest.raises(b.I8Error):
+        b.i8_linear8bit_workspace_layout(4, 4, 16, 100000)

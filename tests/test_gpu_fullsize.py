@@ -2,9 +2,12 @@
 bench.py times (i8_linear8bit_forward with the same max_outlier_cols).
 
 Codes, absmax scales and outlier bitmaps are compared in full (bit-exact);
-int32 accumulators and fp16 outputs on a sample of rows that spans first/last
-tiles and the ragged edge (the oracle evaluates exactly those rows; its
-outlier set is still the union over every row).
+int32 accumulators and fp16 outputs on all rows when a layer has at most 256,
+else on a seeded sample of at least 256 rows (times every output column) that
+also spans the first/last tiles and the ragged edge (the oracle evaluates
+exactly those rows; its outlier set is still the union over every row).  For
+16 tokens or fewer the int32 sums are also taken from the few-token stream-K
+kernel the forward uses (i8_int8_linear_matmul_ws) and compared in full.
 """
 
 import numpy as np
@@ -38,10 +41,13 @@ def host(t):
     return t.cpu().numpy()
 
 
-def sample_rows(M, n=48, seed=0):
+def sample_rows(M, n=256, seed=0):
+    """All rows if M <= n, else n distinct seeded rows plus the tile edges."""
+    if M <= n:
+        return np.arange(M, dtype=np.int64)
     g = np.random.default_rng(seed)
-    fixed = {0, 1, 127, 128, M // 2, M - 1, max(M - 128, 0)}
-    extra = set(g.integers(0, M, size=n).tolist()) if M > n else set(range(M))
+    fixed = {0, 1, 127, 128, 255, 256, M // 2, M - 1, max(M - 128, 0), max(M - 129, 0)}
+    extra = set(g.choice(M, size=n, replace=False).tolist())
     return np.array(sorted(r for r in fixed | extra if 0 <= r < M), dtype=np.int64)
 
 
@@ -79,11 +85,17 @@ def run_layer(i8, key, li, L, X):
     if L.threshold > 0:
         assert np.array_equal(host(bm).view(np.uint32), oracle.outlier_bitmap(rcols, L.K))
     rows = sample_rows(L.M, seed=li)
+    assert len(rows) >= min(L.M, 256)
     # int32 accumulators on the sampled rows (GPU GEMM over the full matrices)
     C = i8.i8_int8_linear_matmul(CA, CB)
     rC = oracle.int8_linear_matmul(rCA[rows], rCB)
     assert np.array_equal(host(C)[rows], rC)
     del C
+    if L.M <= 16:
+        # the few-token stream-K kernel's own int32 sums (split-K partials combined in its workspace)
+        Cd, _ = i8.i8_int8_linear_matmul_ws(CA, CB)
+        assert np.array_equal(host(Cd), rC)
+        del Cd
     # fused forward, as bench.py launches it
     out, ws = i8.i8_linear8bit_forward(dX, CB, SCB, None if b is None else dev(b), L.threshold,
                                        max_outlier_cols=MAX_OUTLIER_COLS)
@@ -115,7 +127,7 @@ def test_llama7b_prefill(i8, key, li):
     run_layer(i8, key, li, L, X)
 
 
-@pytest.mark.parametrize("key,li", layer_params(["C4_t1_o1", "C4_t16_o8", "C4_t4_o0"]))
+@pytest.mark.parametrize("key,li", layer_params(["C4_t1_o1", "C4_t16_o8", "C4_t4_o0", "C4_t4_o8", "C4_t16_o0"]))
 def test_llama70b_decode(i8, key, li):
     L = wl.workloads()[key].layers[li]
     X, _, _, _ = wl.layer_inputs(wl.seed_of(key), li, L)

@@ -305,8 +305,55 @@ def test_selftest_bounded_wait_times_out(i8):
     assert torch.ones(4, device="cuda").sum().item() == 4
 
 
+# ------------------------------------------------------------------ one-launch small forward
+SMALL_SHAPES = [
+    # M, N, K, planted columns, threshold, bias   (all take the one-launch kernel)
+    (16, 1024, 1024, 2, 6.0, True),     # the single-linear workload
+    (1, 1024, 4096, 3, 6.0, False),     # one token, the longest row the kernel takes
+    (5, 300, 272, 4, 6.0, True),        # ragged N (a partial weight tile) and ragged K (a partial box)
+    (16, 4096, 1024, 0, 6.0, True),     # 32 tiles, no outliers
+    (9, 2048, 2064, 40, 6.0, False),    # many outlier columns spread over every stage
+    (12, 512, 1024, 3, 0.0, True),      # threshold 0
+]
+
+
+@pytest.mark.parametrize("M,N,K,n_out,tau,with_bias", SMALL_SHAPES)
+def test_small_forward_against_oracle_and_two_stage(i8, M, N, K, n_out, tau, with_bias):
+    """For few tokens and a small weight the forward is one kernel; the two-stage path
+    (i8_linear8bit_prepare + i8_linear8bit_matmul_dequant) computes the same values with
+    other kernels.  Both are checked against the oracle, and against each other."""
+    X, _ = act(M, K, n_out, mag=(8.0, 60.0), seed=31 + M)
+    W = wl.weight(32 + N, N, K)
+    b = wl.bias(33, N) if with_bias else None
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    dX, dCB, dSCB, db = dev(X), dev(rCB), dev(rSCB), None if b is None else dev(b)
+    out, ws = i8.i8_linear8bit_forward(dX, dCB, dSCB, db, tau)
+    code, count = i8.i8_read_status(ws)
+    _, _, cols = oracle.quantize_rowwise(X, tau)
+    assert code == 0 and count == (len(cols) if tau > 0 else 0)
+    ref = oracle.linear8bit_forward(X, rCB, rSCB, b, tau)
+    assert_close(host(out), ref, "one-launch forward")
+    two = torch.empty_like(out)
+    i8.i8_linear8bit_prepare(dX, dCB, tau, ws, 256)
+    i8.i8_linear8bit_matmul_dequant(dCB, dSCB, db, M, tau, two, ws, 256)
+    assert i8.i8_read_status(ws) == (code, count)
+    assert_close(host(two), ref, "two-stage forward")
+    assert_close(host(out), host(two).astype(np.float64), "one-launch vs two-stage")
+
+
+def test_small_forward_repeat_is_deterministic(i8):
+    X, _ = act(16, 1024, 2, seed=40)
+    W = wl.weight(41, 1024, 1024)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    dX, dCB, dSCB = dev(X), dev(rCB), dev(rSCB)
+    a, ws = i8.i8_linear8bit_forward(dX, dCB, dSCB, None, 6.0)
+    for _ in range(3):
+        b, _ = i8.i8_linear8bit_forward(dX, dCB, dSCB, None, 6.0, workspace=ws)
+        assert torch.equal(a, b)
+
+
 # ------------------------------------------------------------------ CUDA graph capture
-@pytest.mark.parametrize("M,N,K,n_out", [(256, 512, 1024, 3), (4, 4096, 8192, 5)])
+@pytest.mark.parametrize("M,N,K,n_out", [(256, 512, 1024, 3), (4, 4096, 8192, 5), (16, 1024, 1024, 2)])
 def test_forward_cuda_graph_replay(i8, M, N, K, n_out):
     """The forward never waits for the host: it can be captured once and replayed on new
     inputs (a different outlier set each time), the outlier columns being found on the device."""
@@ -408,8 +455,9 @@ MSHAPES = [
     (300, 1040, (520, 264, 1040), 3, 6.0),    # prefill, few outlier columns
     (512, 1024, (4096, 4096), 40, 6.0),       # prefill, > 16 columns: tcgen05 fp16 outlier path
     (300, 1040, (520, 264), 3, 0.0),          # threshold 0
-    (7, 2064, (1000, 272, 4096), 5, 6.0),     # few tokens: one preparation, three decode GEMMs
-    (16, 4096, (4096, 1024), 40, 6.0),        # few tokens, many outlier columns
+    (7, 2064, (1000, 272, 4096), 5, 6.0),     # few tokens: two one-launch weights, one decode GEMM
+    (16, 4096, (4096, 1024), 40, 6.0),        # few tokens, many outlier columns (one of each path)
+    (5, 1024, (1024, 512, 264), 3, 6.0),      # few tokens, every weight one-launch
 ]
 
 

@@ -70,6 +70,11 @@ def test_nearest_rank_percentiles():
     assert bench.nearest_rank([3.0], (0.1, 0.5, 0.9)) == [3.0, 3.0, 3.0]
     xs = [float(x) for x in range(11, 0, -1)]          # 11 .. 1, unsorted input
     assert bench.nearest_rank(xs, (0.0, 0.1, 0.5, 0.9, 1.0)) == [1.0, 2.0, 6.0, 10.0, 11.0]
+    # the ceil(p * n)-th smallest value (1-based): for n = 4 the median is the 2nd value, for
+    # n = 20 the 10th percentile is the 2nd and the 90th the 18th
+    assert bench.nearest_rank([4.0, 1.0, 3.0, 2.0], (0.5,)) == [2.0]
+    ys = [float(x) for x in range(1, 21)]
+    assert bench.nearest_rank(ys, (0.1, 0.9)) == [2.0, 18.0]
 
 
 def test_reference_arm_reports_on_rank_zero_only():
@@ -90,3 +95,74 @@ def test_reference_arm_reports_on_rank_zero_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+# ------------------------------------------------------------------ column-parallel split
+def _column_worker(rank, world, port, queue):
+    """One rank of the column split, on CPU: the oracle stands in for the rank's local
+    forward (the CUDA forward of the same rows is checked against it on the GPU); the
+    partitioning and the all-gather are the package's own."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from int8_mixed_precision_vectorwise_b200 import column_parallel as cp
+    from int8_mixed_precision_vectorwise_b200 import workloads as wl
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        M, K, N = 9, 64, 40
+        X, _ = wl.activation(wl.BASE_SEED + 5, M, K, 2, (20.0, 40.0))
+        CB, SCB = oracle.quantize_weight_rowwise(wl.weight(6, N, K))
+        bias = wl.bias(7, N)
+        n0, n1 = cp.shard_range(N, world, rank)
+        local = oracle.linear8bit_forward(X, CB[n0:n1], SCB[n0:n1], bias[n0:n1], 6.0)
+        G = cp.gather_column_blocks(torch.from_numpy(local), world)
+        queue.put((rank, (n0, n1), G.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_column_split_two_gloo_ranks():
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    from int8_mixed_precision_vectorwise_b200 import workloads as wl
+    world = 2
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_column_worker, args=(r, world, port, queue)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        rank, rng, G = queue.get(timeout=120)
+        got[rank] = (rng, G)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # the shards tile the output columns in rank order
+    assert [got[r][0] for r in range(world)] == [(0, 20), (20, 40)]
+    # every rank holds the same gather: rank-major blocks; laid out as out[m, p*Np + j] = G[p, m, j]
+    # it is the whole layer's output, bit for bit (the oracle treats each output column alone)
+    assert np.array_equal(got[0][1].view(np.uint16), got[1][1].view(np.uint16))
+    G = got[0][1]
+    P, M, Np = G.shape
+    out = np.transpose(G, (1, 0, 2)).reshape(M, P * Np)
+    X, _ = wl.activation(wl.BASE_SEED + 5, 9, 64, 2, (20.0, 40.0))
+    CB, SCB = oracle.quantize_weight_rowwise(wl.weight(6, 40, 64))
+    ref = oracle.linear8bit_forward(X, CB, SCB, wl.bias(7, 40), 6.0)
+    assert np.array_equal(out.view(np.uint16), ref.view(np.uint16))
+
+
+def test_shard_range_rules():
+    sys.path.insert(0, ROOT)
+    from int8_mixed_precision_vectorwise_b200 import column_parallel as cp
+    assert [cp.shard_range(28672, 8, r) for r in (0, 7)] == [(0, 3584), (25088, 28672)]
+    assert cp.shard_range(5, 1, 0) == (0, 5)
+    with pytest.raises(ValueError):
+        cp.shard_range(10, 3, 0)
+    with pytest.raises(ValueError):
+        cp.shard_range(10, 2, 2)
