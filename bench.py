@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-other", action="store_true", help="skip the single-linear, OPT MLP and outlier sweep")
     ap.add_argument("--no-shared", action="store_true", help="skip the shared-input layer step")
+    ap.add_argument("--no-quant", action="store_true", help="skip the quantiser roofline")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows per linear in the CPU oracle sample")
     return ap.parse_args()
 
@@ -165,9 +166,11 @@ def job_throughput(ops_per_step: float, steps: int, world: int, ms: float) -> fl
 
 
 def nearest_rank(xs, ps):
-    """Nearest-rank percentiles (p in [0, 1]) of a non-empty sample."""
+    """Nearest-rank percentiles (p in [0, 1]) of a non-empty sample: the ceil(p * n)-th
+    smallest value (the smallest one for p = 0)."""
+    import math
     v = sorted(xs)
-    return [v[min(len(v) - 1, max(0, int(round(p * (len(v) - 1)))))] for p in ps]
+    return [v[min(len(v) - 1, max(0, math.ceil(p * len(v)) - 1))] for p in ps]
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -187,14 +190,23 @@ def cpu_oracle_steps(layers_np, rows: int, steps: int, min_seconds: float = 0.0)
     return times, ops
 
 
+def decode_bytes(L) -> int:
+    """Algorithmic bytes of one few-token forward: the int8 weight, its scales, X and out."""
+    return L.N * L.K + 4 * L.N + 2 * L.M * L.K + 2 * L.M * L.N
+
+
 def measure_decode(i8, torch, dev, st, world, dist, reps: int = 20):
-    """Whole forward (quantise + outlier prepare + decode GEMM) per call on the
-    Llama-70B FFN shapes; weights (235 MB each, > L2) stream from HBM every call."""
+    """Every point of the decode grid (tokens {1, 4, 16} x outlier columns {0, 1, 8}) on both
+    Llama-70B FFN shapes.  Weights (235 MB each, > L2) stream from HBM every call.  Per point:
+    the whole forward (preparation + few-token GEMM, launched as in production, `reps`
+    back-to-back calls), then a second pass with events between the two kernels, which gives
+    the preparation alone and the GEMM alone (each then starts without the other's overlap)."""
     W = wl.workloads()
     points = []
     hbm = (measured_peaks() or {}).get("hbm_gbs", 6650.0)
     weights = {}
-    for key in ("C4_t1_o1", "C4_t16_o8"):
+    keys = [f"C4_t{t}_o{o}" for t in (1, 4, 16) for o in (0, 1, 8)]
+    for key in keys:
         for li, L in enumerate(W[key].layers):
             wk = (L.N, L.K)
             if wk not in weights:
@@ -207,32 +219,104 @@ def measure_decode(i8, torch, dev, st, world, dist, reps: int = 20):
             out = torch.empty((L.M, L.N), dtype=torch.float16, device=dev)
             ws = torch.empty((i8.i8_linear8bit_workspace_size(L.M, L.N, L.K, MAX_OUTLIER_COLS),),
                              dtype=torch.uint8, device=dev)
-            for _ in range(3):
+
+            def fwd():
                 i8.i8_linear8bit_forward(dX, CB, SCB, None, L.threshold, out=out, workspace=ws,
                                          max_outlier_cols=MAX_OUTLIER_COLS)
+            for _ in range(3):
+                fwd()
             if world > 1:
                 dist.barrier()
             torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(st)
             for _ in range(reps):
-                i8.i8_linear8bit_forward(dX, CB, SCB, None, L.threshold, out=out, workspace=ws,
-                                         max_outlier_cols=MAX_OUTLIER_COLS)
+                fwd()
             e1.record(st)
+            torch.cuda.synchronize(dev)
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+            for r in range(reps):
+                ev[r][0].record(st)
+                i8.i8_linear8bit_prepare(dX, CB, L.threshold, ws, MAX_OUTLIER_COLS)
+                ev[r][1].record(st)
+                i8.i8_linear8bit_matmul_dequant(CB, SCB, None, L.M, L.threshold, out, ws, MAX_OUTLIER_COLS)
+                ev[r][2].record(st)
             torch.cuda.synchronize(dev)
             code, _ = i8.i8_read_status(ws)
             if code != 0:
                 raise RuntimeError(f"decode status {i8.STATUS.get(code, code)}")
             us = e0.elapsed_time(e1) / reps * 1e3
-            byts = L.N * L.K + 4 * L.N + 2 * L.M * L.K + 2 * L.M * L.N
-            gbs = byts / us / 1e3
+            prep_us = sum(a.elapsed_time(b) for a, b, _ in ev) / reps * 1e3
+            gemm_us = sum(b.elapsed_time(c) for _, b, c in ev) / reps * 1e3
+            gbs = decode_bytes(L) / us / 1e3
             points.append({"shape": f"{L.M}x{L.K}->{L.N}", "tokens": L.M, "outlier_cols": L.n_out,
-                           "us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4)})
+                           "us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                           "prep_alone_us": round(prep_us, 2), "gemm_alone_us": round(gemm_us, 2),
+                           "gemm_alone_frac": round(decode_bytes(L) / gemm_us / 1e3 / hbm, 4)})
     best = max(points, key=lambda q: q["GB/s"])
+    worst = min(points, key=lambda q: q["GB/s"])
     return {"metric": "decode weight-read GB/s (whole forward per call)", "peak_gbs": hbm,
             "peak_source": "of measured hbm_gbs" if measured_peaks() else "of fallback",
             "bytes": "N*K + 4N + 2MK + 2MN per call", "points": points,
-            "best_GB/s": best["GB/s"], "best_frac": best["frac"]}
+            "best_GB/s": best["GB/s"], "best_frac": best["frac"],
+            "worst_GB/s": worst["GB/s"], "worst_frac": worst["frac"]}
+
+
+def measure_quant(i8, torch, dev, st, world, dist, reps: int = 40):
+    """The fused quantiser alone on the Llama-7B prefill activation shapes (4096 tokens x 4096
+    and x 11008 features).  Launched with threshold 0, i8_quantize_rowwise is exactly one
+    quantiser kernel; with threshold 6 it adds the bitmap memset and the column-zeroing kernel.
+    Inputs rotate over enough copies (> 2 x L2) that every call reads X from HBM.
+    Algorithmic bytes per call: 2MK (X) + MK (codes) + 4M (scales) + K/8 (bitmap)."""
+    hbm = (measured_peaks() or {}).get("hbm_gbs", 6650.0)
+    res = []
+    for M, K in ((4096, 4096), (4096, 11008)):
+        X, _ = wl.activation(wl.BASE_SEED + 900 + K, M, K, round(0.001 * K), (20.0, 60.0))
+        per = 3 * M * K
+        n = max(4, int(np.ceil(2.5 * 126e6 / per)))
+        Xs = [torch.from_numpy(X).to(dev) for _ in range(n)]
+        CAs = [torch.empty((M, K), dtype=torch.int8, device=dev) for _ in range(n)]
+        SCA = torch.empty((M,), dtype=torch.float32, device=dev)
+        bm = torch.empty(((K + 31) // 32,), dtype=torch.int32, device=dev)
+        row = {"shape": f"{M}x{K}"}
+        for tau in (0.0, 6.0):
+            for i in range(n):
+                i8.i8_quantize_rowwise(Xs[i], tau, CA=CAs[i], SCA=SCA, bitmap=bm)
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for r in range(reps):
+                i8.i8_quantize_rowwise(Xs[r % n], tau, CA=CAs[r % n], SCA=SCA, bitmap=bm)
+            e1.record(st)
+            torch.cuda.synchronize(dev)
+            us = e0.elapsed_time(e1) / reps * 1e3
+            gbs = (2 * M * K + M * K + 4 * M + K / 8) / us / 1e3
+            tag = "kernel" if tau == 0.0 else "op_tau6"
+            row.update({f"{tag}_us": round(us, 2), f"{tag}_GB/s": round(gbs, 1), f"{tag}_frac": round(gbs / hbm, 4)})
+        res.append(row)
+        del Xs, CAs
+    return {"kernel": "k_quant_rows", "peak_gbs": hbm,
+            "peak_source": "of measured hbm_gbs" if measured_peaks() else "of fallback",
+            "bytes": "2MK + MK + 4M + K/8 per call",
+            "timing": f"CUDA events over {reps} back-to-back calls, inputs rotated over > 2 x L2",
+            "kernel_us": "threshold 0: the quantiser kernel alone; op_tau6: memset + quantiser + column zeroing",
+            "points": res}
+
+
+def cpu_per_config(layers_by_key, rows: int, min_seconds: float):
+    """The oracle on a bounded row sample of each other workload family, one timing each."""
+    res = {}
+    for key, (layers_np, byts) in layers_by_key.items():
+        times, ops = cpu_oracle_steps(layers_np, rows, 1, min_seconds=min_seconds)
+        t = sum(times) / len(times)
+        n_rows = [min(rows, X.shape[0]) for X, *_ in layers_np]
+        e = {"TOPS": ops / t / 1e12, "sample_rows": n_rows, "passes": len(times), "s_per_pass": t}
+        if byts is not None:
+            e["GB/s"] = byts / t / 1e9
+        res[key] = e
+    return res
 
 
 def measure_backward(i8, torch, dev, st, world, dist, reps: int = 20):
@@ -457,7 +541,10 @@ def cpu_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_layers(W: wl.Workload, seed: int):
+def oracle_layers(W: wl.Workload, seed: int, weight_rows=None):
+    """Oracle operands of every linear of a workload.  `weight_rows` keeps only the first
+    rows of each weight (a sample of the output columns; the outlier set and row scales
+    still come from the whole of X)."""
     import oracle
     out = []
     for li, L in enumerate(W.layers):
@@ -465,6 +552,9 @@ def oracle_layers(W: wl.Workload, seed: int):
         if X is None:   # chained input: the oracle feeds itself (ReLU of its own previous output)
             pX, pCB, pSCB, pb, ptau = out[-1]
             X = np.maximum(oracle.linear8bit_forward(pX, pCB, pSCB, pb, ptau), np.float16(0))
+        if weight_rows is not None:
+            Wt = Wt[:weight_rows]
+            b = None if b is None else b[:weight_rows]
         CB, SCB = oracle.quantize_weight_rowwise(Wt)
         out.append((X, CB, SCB, b, L.threshold))
     return out
@@ -679,6 +769,11 @@ def run_ours(args):
     if not args.no_other:
         other_wl = measure_other(i8, torch, dev, st, world, dist)
 
+    # ---- the quantiser alone (HBM roofline)
+    quant = None
+    if not args.no_quant:
+        quant = measure_quant(i8, torch, dev, st, world, dist)
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -688,6 +783,23 @@ def run_ours(args):
                "kind": "oracle",
                "sample": f"first {args.cpu_rows} rows of each of the {len(layers_np)} linears, "
                          f"{len(times)} passes ({sum(times):.1f} s)"}
+        # the other workload families, each on a bounded sample (first 64 activation rows; the
+        # decode point on its 16 tokens and the first 2048 rows of each weight, bytes counted
+        # for that sample)
+        Wall = wl.workloads()
+        dec = Wall["C4_t16_o8"]
+        dec_np = oracle_layers(dec, wl.seed_of("C4_t16_o8"), weight_rows=2048)
+        dec_bytes = sum(CB.shape[0] * CB.shape[1] + 4 * CB.shape[0] + 2 * X.shape[0] * X.shape[1]
+                        + 2 * X.shape[0] * CB.shape[0] for X, CB, *_ in dec_np)
+        per = {
+            "C1_single_linear": (oracle_layers(Wall["C1"], wl.seed_of("C1")), None),
+            "C2_opt350m_mlp": (oracle_layers(Wall["C2"], wl.seed_of("C2")), None),
+            "C4_llama70b_decode_t16_o8": (dec_np, dec_bytes),
+            "C5_llama13b_mlp_f0.01_t6": (oracle_layers(Wall["C5_f0.01_t6"], wl.seed_of("C5_f0.01_t6")), None),
+        }
+        cpu["per_config"] = cpu_per_config(per, 64, min_seconds=1.5)
+        cpu["per_config_sample"] = ("first 64 activation rows of every linear (C1: all 16; C4: its 16 tokens "
+                                    "and the first 2048 rows of each weight), repeated for >= 1.5 s")
 
     if world > 1:
         dist.barrier()
@@ -736,10 +848,22 @@ def run_ours(args):
                      "gemm_ms_per_step": gemm_ms / K, "gemm_share_of_step": gemm_ms / ms_instr,
                      "gemm_ms_per_step_p10_p50_p90": nearest_rank(gemm_step_ms, (0.1, 0.5, 0.9)),
                      "gemm_timing": "CUDA events around each GEMM launch in a second pass of the same "
-                                    f"{K} steps ({ms_instr / K:.4f} ms per instrumented step)"},
+                                    f"{K} steps ({ms_instr / K:.4f} ms per instrumented step)",
+                     "quant": None if quant is None else {
+                         "kernel": quant["kernel"], "bytes": quant["bytes"], "peak_gbs": quant["peak_gbs"],
+                         "points": [[q["shape"], q["kernel_us"], q["kernel_GB/s"], q["kernel_frac"]]
+                                    for q in quant["points"]],
+                         "columns": ["shape", "us", "GB/s", "frac"]},
+                     "decode": None if decode is None else {
+                         "kernel": "k_decode_prep + k_gemm_i8_decode (whole forward)", "bytes": decode["bytes"],
+                         "peak_gbs": decode["peak_gbs"],
+                         "points": [[q["tokens"], q["outlier_cols"], q["shape"], q["us"], q["GB/s"], q["frac"]]
+                                    for q in decode["points"]],
+                         "columns": ["tokens", "outlier_cols", "shape", "us", "GB/s", "frac"]}},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "decode": decode,
+        "quant": quant,
         "backward": backward,
         "other_workloads": other_wl,
         "shared_inputs": shared,
