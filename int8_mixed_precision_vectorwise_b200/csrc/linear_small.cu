@@ -45,6 +45,7 @@ constexpr int LSTAGE = LSB * LBOX;            // 32 KB
 constexpr int LRS = 4;                        // ring stages
 constexpr int LCA_BOX = LT * 128;             // one 128-byte-deep box of the 16 code rows: 2 KB
 constexpr int LTHREADS = 256;
+constexpr int LPU = 8;                        // X vectors per thread in flight while quantising
 constexpr uint32_t LTMEM_COLS = 32;
 constexpr unsigned kAllLanes = 0xffffffffu;
 
@@ -136,37 +137,53 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   }
 
   // ---------------------------------------------------------------- quantise X (all threads)
+  // Items (row, 8-column vector) in chunks of LPU per thread: all LPU loads of
+  // a chunk are issued before any is used.  When X fits in one chunk it stays
+  // in registers for pass 2; otherwise pass 2 reads each chunk again (from L1/L2).
   const int items = M * nvec;
-  for (int base = 0; base < items; base += LTHREADS) {   // pass 1: row maxima below the threshold, column flags
-    const int it = base + tid;                             // (uniform trip count: whole warps vote below)
-    const bool valid = it < items;
-    const int r = valid ? it / nvec : -1;
-    float keep = 0.f;
-    if (valid) {
-      const int v = it - r * nvec;
-      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + v);
-      const __half2* h = reinterpret_cast<const __half2*>(&xv);
-      const __half2 m2 = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
-      const float vmax = fmaxf(__low2float(m2), __high2float(m2));
-      if (!use_tau || vmax < tau) {
-        keep = vmax;
-      } else {
-        uint32_t big = 0;
+  const bool one_chunk = items <= LPU * LTHREADS;
+  uint4 xv[LPU];
+  for (int base = 0; base < items; base += LPU * LTHREADS) {   // pass 1: row maxima below the threshold, column flags
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(h[e]);
-          const float a0 = fabsf(f.x), a1 = fabsf(f.y);
-          if (a0 >= tau) big |= 1u << (2 * e); else keep = fmaxf(keep, a0);
-          if (a1 >= tau) big |= 2u << (2 * e); else keep = fmaxf(keep, a1);
-        }
-        atomicOr(sbm + (v >> 2), big << ((v & 3) * 8));
+    for (int u = 0; u < LPU; ++u) {
+      const int it = base + u * LTHREADS + tid;
+      xv[u] = make_uint4(0, 0, 0, 0);
+      if (it < items) {
+        const int r = it / nvec;
+        xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + (it - r * nvec));
       }
     }
-    // lanes of the same row combine their maxima (non-negative floats order like their
-    // bits); one shared atomic per row and warp
-    const unsigned same = __match_any_sync(kAllLanes, r);
-    const unsigned mx = __reduce_max_sync(same, __float_as_uint(keep));
-    if (valid && lane == __ffs(same) - 1) atomicMax(s_rowmax + r, mx);
+#pragma unroll
+    for (int u = 0; u < LPU; ++u) {   // (uniform trip count: whole warps vote below)
+      const int it = base + u * LTHREADS + tid;
+      const bool valid = it < items;
+      const int r = valid ? it / nvec : -1;
+      float keep = 0.f;
+      if (valid) {
+        const int v = it - r * nvec;
+        const __half2* h = reinterpret_cast<const __half2*>(&xv[u]);
+        const __half2 m2 = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])), __hmax2(__habs2(h[2]), __habs2(h[3])));
+        const float vmax = fmaxf(__low2float(m2), __high2float(m2));
+        if (!use_tau || vmax < tau) {
+          keep = vmax;
+        } else {
+          uint32_t big = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            const float a0 = fabsf(f.x), a1 = fabsf(f.y);
+            if (a0 >= tau) big |= 1u << (2 * e); else keep = fmaxf(keep, a0);
+            if (a1 >= tau) big |= 2u << (2 * e); else keep = fmaxf(keep, a1);
+          }
+          atomicOr(sbm + (v >> 2), big << ((v & 3) * 8));
+        }
+      }
+      // lanes of the same row combine their maxima (non-negative floats order like their
+      // bits); one shared atomic per row and warp
+      const unsigned same = __match_any_sync(kAllLanes, r);
+      const unsigned mx = __reduce_max_sync(same, __float_as_uint(keep));
+      if (valid && lane == __ffs(same) - 1) atomicMax(s_rowmax + r, mx);
+    }
   }
   __syncthreads();
   if (tid < LT) {
@@ -175,29 +192,43 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     s_sa[tid] = amax * (1.0f / 16129.0f);
   }
   __syncthreads();
-  for (int it = tid; it < items; it += LTHREADS) {   // pass 2: codes into the swizzled K-major tile
-    const int r = it / nvec, v = it - r * nvec;
-    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + v);
-    const float rs = s_r[r];
-    const uint32_t fl = (sbm[v >> 2] >> ((v & 3) * 8)) & 0xffu;
-    const __half2* h = reinterpret_cast<const __half2*>(&xv);
-    uint32_t w[2];
+  for (int base = 0; base < items; base += LPU * LTHREADS) {   // pass 2: codes into the swizzled K-major tile
+    if (!one_chunk) {
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      const float2 a = __half22float2(h[2 * p]);
-      const float2 b = __half22float2(h[2 * p + 1]);
-      const uint32_t lo = __byte_perm(small_code(a.x, rs), small_code(a.y, rs), 0x0040);
-      const uint32_t hi = __byte_perm(small_code(b.x, rs), small_code(b.y, rs), 0x0040);
-      w[p] = __byte_perm(lo, hi, 0x5410);
+      for (int u = 0; u < LPU; ++u) {
+        const int it = base + u * LTHREADS + tid;
+        if (it < items) {
+          const int r = it / nvec;
+          xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + (it - r * nvec));
+        }
+      }
     }
-    if (fl) {  // outlier columns carry code 0
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (fl & (1u << e)) w[e >> 2] &= ~(0xffu << ((e & 3) * 8));
+    for (int u = 0; u < LPU; ++u) {
+      const int it = base + u * LTHREADS + tid;
+      if (it >= items) break;
+      const int r = it / nvec, v = it - r * nvec;
+      const float rs = s_r[r];
+      const uint32_t fl = (sbm[v >> 2] >> ((v & 3) * 8)) & 0xffu;
+      const __half2* h = reinterpret_cast<const __half2*>(&xv[u]);
+      uint32_t w[2];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float2 a = __half22float2(h[2 * p]);
+        const float2 b = __half22float2(h[2 * p + 1]);
+        const uint32_t lo = __byte_perm(small_code(a.x, rs), small_code(a.y, rs), 0x0040);
+        const uint32_t hi = __byte_perm(small_code(b.x, rs), small_code(b.y, rs), 0x0040);
+        w[p] = __byte_perm(lo, hi, 0x5410);
+      }
+      if (fl) {  // outlier columns carry code 0
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (fl & (1u << e)) w[e >> 2] &= ~(0xffu << ((e & 3) * 8));
+      }
+      // byte kk = 8v of row r: box kk / 128, 16-byte chunk q = (kk % 128) / 16 stored at q ^ (r % 8)
+      const int kk = 8 * v, box = kk >> 7, q = (kk & 127) >> 4;
+      *reinterpret_cast<uint2*>(ca + box * LCA_BOX + r * 128 + ((q ^ (r & 7)) << 4) + (kk & 15)) = make_uint2(w[0], w[1]);
     }
-    // byte kk = 8v of row r: box kk / 128, 16-byte chunk q = (kk % 128) / 16 stored at q ^ (r % 8)
-    const int kk = 8 * v, box = kk >> 7, q = (kk & 127) >> 4;
-    *reinterpret_cast<uint2*>(ca + box * LCA_BOX + r * 128 + ((q ^ (r & 7)) << 4) + (kk & 15)) = make_uint2(w[0], w[1]);
   }
   if (warp == 0) {   // the sorted outlier list (ascending columns)
     const int per = (nwords + 31) / 32;

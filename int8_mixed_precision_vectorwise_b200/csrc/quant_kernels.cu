@@ -43,15 +43,17 @@ __device__ __forceinline__ void scan8(const uint4& v, float tau, bool use_tau, f
   }
 }
 
-// int8 code of x * r, rounded to nearest even.  The convert saturates to
-// [-128, 127]; that equals clipping to [-127, 127] for every element kept on
-// the int8 path (|x| <= amax, so |x * r| <= 127 * (1 + 2^-23)).  Elements at or
-// above the threshold may saturate to -128, but their columns are outlier
-// columns, whose codes are zeroed before use.
-__device__ __forceinline__ uint32_t code_s8(float x, float r) {
-  uint32_t q;
-  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(x, r)));
-  return q;
+// int8 code of x * r, rounded to nearest even, in the low byte of the result.
+// t = fl32(x * r) is rounded once more by adding 1.5 * 2^23: for |t| <= 2^22
+// the sum lies in [2^23, 2^24), where fp32 holds exactly the integers, so IEEE
+// round-to-nearest-even makes it 1.5 * 2^23 + rne(t), and the low byte of its
+// bit pattern is rne(t) as a two's-complement byte (the constant's low 22 bits
+// are 0).  This is the reading's code for every element kept on the int8 path
+// (|x| <= amax, so |t| <= 127 * (1 + 2^-23) and no clamp is reached).  Larger
+// t only occur at or above the threshold, in outlier columns, whose codes are
+// zeroed before use.  Two FMA-pipe operations instead of a conversion.
+__device__ __forceinline__ uint32_t code_rne(float x, float r) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, r), 12582912.0f));
 }
 
 // 8 fp16 values -> 8 int8 codes packed little-endian.
@@ -62,8 +64,8 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float r) {
   for (int p = 0; p < 2; ++p) {
     const float2 a = __half22float2(h[2 * p]);
     const float2 b = __half22float2(h[2 * p + 1]);
-    const uint32_t lo = __byte_perm(code_s8(a.x, r), code_s8(a.y, r), 0x0040);
-    const uint32_t hi = __byte_perm(code_s8(b.x, r), code_s8(b.y, r), 0x0040);
+    const uint32_t lo = __byte_perm(code_rne(a.x, r), code_rne(a.y, r), 0x0040);
+    const uint32_t hi = __byte_perm(code_rne(b.x, r), code_rne(b.y, r), 0x0040);
     w[p] = __byte_perm(lo, hi, 0x5410);
   }
   return make_uint2(w[0], w[1]);
@@ -171,30 +173,32 @@ __global__ void __launch_bounds__(256, (VPT > 8 ? 1 : 5)) k_quant_rows(const __h
 // Each CTA (one per SM) owns a contiguous range of rows.  Lane 0 of warp 0
 // streams whole rows of X into a ring of shared-memory slots with 1-D bulk
 // copies, so up to `slots` rows (~200 KB) per SM are in flight while rows are
-// being quantised; a slot is refilled as soon as the row in it is done.  The
-// other 8 warps quantise one row at a time together, from shared memory:
-// absmax over the row (elements at or above the threshold left out and marked
-// in the CTA's outlier bitmap), one fp32 division, codes written with 8-byte
-// coalesced stores.  Every wait is bounded; a timeout sets *status (when
-// given) and all warps leave together (the per-row barrier also ORs the
-// warps' failures), the producer first waiting, bounded, for its copies.
-constexpr int kRingConsumers = 256;  // threads that quantise a row together
-constexpr int kRingThreads = 32 + kRingConsumers;
+// being quantised; a slot is refilled as soon as the row in it is done.  Each
+// of the other `nwc` warps quantises its own rows (row j of the range goes to
+// warp j % nwc) from shared memory, with warp-level reductions only, so many
+// rows are in progress at once.  `slots` is a multiple of `nwc`, so a slot
+// only ever holds rows of one warp, which takes them in order: no wait can
+// run a whole phase ahead of the slot's barrier.  Per row: absmax over the row (elements at or above the
+// threshold left out and marked in the CTA's outlier bitmap), one fp32
+// division, codes written with 8-byte coalesced stores.  Every wait is
+// bounded; a timeout sets *status (when given), the warps leave their loops
+// and the producer first waits, bounded, for its copies.
+constexpr int kRingWarps = 8;        // most consumer warps, one row each at a time
+constexpr int kRingThreads = 32 * (1 + kRingWarps);
 constexpr int kRingMaxSlots = 32;
 constexpr int kRingSlotBudget = 200 * 1024;
 
 __global__ void __launch_bounds__(kRingThreads, 1)
     k_quant_rows_ring(const __half* __restrict__ X, int M, int K, float tau, int8_t* __restrict__ CA,
                       float* __restrict__ SCA, uint32_t* __restrict__ bitmap, int rows_per_cta, int slots,
-                      uint32_t* status, uint64_t limit_ns) {
+                      int nwc, uint32_t* status, uint64_t limit_ns) {
   extern __shared__ __align__(128) uint8_t rsm[];
   const int row_bytes = 2 * K;
   uint8_t* ring = rsm;
   uint64_t* full = reinterpret_cast<uint64_t*>(rsm + static_cast<size_t>(slots) * row_bytes);
   uint64_t* empty = full + slots;
-  float* red = reinterpret_cast<float*>(empty + slots);  // [2][8]: row parity x consumer warp
-  volatile int* s_abort = reinterpret_cast<volatile int*>(red + 16);
-  uint32_t* sbm = reinterpret_cast<uint32_t*>(red + 20);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(empty + slots);
+  uint32_t* sbm = reinterpret_cast<uint32_t*>(empty + slots) + 4;
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = blockIdx.x * rows_per_cta;
@@ -204,7 +208,7 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < slots; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kRingConsumers / 32);
+      mbar_init(&empty[s], 1);  // the warp that quantised the slot's row
     }
     *s_abort = 0;
     fence_barrier_init();
@@ -234,31 +238,25 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- consumers
-    const int t = threadIdx.x - 32, cw = warp - 1;
-    for (int j = 0; j < n; ++j) {
+    for (int j = warp - 1; warp <= nwc && j < n; j += nwc) {
       const int s = j % slots;
-      const uint32_t parity = static_cast<uint32_t>(j / slots) & 1u;
       int ok = 0;
-      if (lane == 0) ok = mbar_wait_bounded(&full[s], parity, s_abort, status, limit_ns) ? 1 : 0;
-      ok = __shfl_sync(kFull, ok, 0);
+      if (lane == 0) ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / slots) & 1u, s_abort, status, limit_ns);
+      if (!__shfl_sync(kFull, ok, 0)) break;
       const uint4* v = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(s) * row_bytes);
       float amax = 0.f;
-      if (ok)
-        for (int vi = t; vi < nvec; vi += kRingConsumers) fold8(v[vi], vi, tau, use_tau, amax, sbm);
+#pragma unroll 4
+      for (int vi = lane; vi < nvec; vi += 32) fold8(v[vi], vi, tau, use_tau, amax, sbm);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-      if (lane == 0) red[(j & 1) * 8 + cw] = amax;
-      if (named_bar_any(1, kRingConsumers, !ok)) break;  // every consumer warp leaves at the same row
-      amax = red[(j & 1) * 8];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[(j & 1) * 8 + w]);
       const float r = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
       const int row = r0 + j;
-      if (t == 0) SCA[row] = amax;
+      if (lane == 0) SCA[row] = amax;
       uint2* cr = reinterpret_cast<uint2*>(CA + static_cast<size_t>(row) * K);
-      for (int vi = t; vi < nvec; vi += kRingConsumers) cr[vi] = quant8(v[vi], r);
+#pragma unroll 4
+      for (int vi = lane; vi < nvec; vi += 32) cr[vi] = quant8(v[vi], r);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the slot
+      if (lane == 0) mbar_arrive(&empty[s]);  // the slot may be refilled
     }
   }
   __syncthreads();
@@ -582,8 +580,10 @@ cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* 
   if (K >= 1024 && K <= 16384 && num_sms > 0) {
     // rows of 2 KB .. 32 KB: the persistent ring kernel, one CTA per SM
     const int row_bytes = 2 * K;
-    const int slots = std::min(kRingMaxSlots, kRingSlotBudget / row_bytes);
-    const size_t ring_smem = static_cast<size_t>(slots) * row_bytes + static_cast<size_t>(slots) * 16 + 20 * 4 +
+    // consumer warps, and slots rounded down to a multiple of them (each warp its own slots)
+    const int nwc = std::min(kRingWarps, std::min(kRingMaxSlots, kRingSlotBudget / row_bytes));
+    const int slots = (std::min(kRingMaxSlots, kRingSlotBudget / row_bytes) / nwc) * nwc;
+    const size_t ring_smem = static_cast<size_t>(slots) * row_bytes + static_cast<size_t>(slots) * 16 + 16 +
                              static_cast<size_t>((K + 31) / 32) * 4;
     static std::atomic<bool> attr_done[64];
     int dev = 0;
@@ -598,7 +598,7 @@ cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* 
     const int rows_per_cta = (M + grid - 1) / grid;
     grid = (M + rows_per_cta - 1) / rows_per_cta;
     k_quant_rows_ring<<<grid, kRingThreads, ring_smem, st>>>(X, M, K, tau, CA, SCA, bitmap, rows_per_cta, slots,
-                                                              status, limit_ns);
+                                                              nwc, status, limit_ns);
     return cudaGetLastError();
   }
   // One row per group of threads with the row in registers (one pass over X),

@@ -228,3 +228,19 @@ def test_workspace_layout_matches_size():
         b.i8_linear8bit_workspace_layout(0, 4, 16, 8)
     with pytest.raises(b.I8Error):
         b.i8_linear8bit_workspace_layout(4, 4, 16, 100000)
+
+
+def test_int8_rounding_by_added_constant_is_round_half_even():
+    """The quantiser rounds t = fl32(x * r) by adding 1.5 * 2^23 in fp32 and keeping the low
+    byte of the sum's bits.  That byte must be rne(t) (two's complement) for every |t| <= 128:
+    ties on a 2^-12 grid, their fp32 neighbours, and random values."""
+    import numpy as np
+    grid = (np.arange(-128 * 4096, 128 * 4096 + 1, dtype=np.float64) / 4096).astype(np.float32)
+    ties = (np.arange(-128, 128, dtype=np.float32) + np.float32(0.5))
+    near = np.concatenate([np.nextafter(ties, np.float32(-np.inf)), np.nextafter(ties, np.float32(np.inf))])
+    rnd = np.random.default_rng(0).uniform(-128, 128, 1_000_000).astype(np.float32)
+    t = np.concatenate([grid, ties, near, rnd, np.float32([0.0, -0.0])])
+    s = (t + np.float32(12582912.0)).astype(np.float32)     # one fp32 addition, round to nearest even
+    low = (s.view(np.uint32) & np.uint32(0xFF)).astype(np.uint8).view(np.int8)
+    want = np.rint(t.astype(np.float64))                     # numpy rint: half to even
+    assert np.array_equal(low.astype(np.int64), ((want.astype(np.int64) + 128) % 256) - 128)
