@@ -25,8 +25,12 @@ notes):
       midpoints m_i = fl32((v_i + v_{i+1}) / 2) strictly below y, i.e. the
       nearest level with ties to the lower one.  Byte j of a row holds the codes
       of elements 2j (low nibble) and 2j + 1 (high nibble).
-* R13 dequantisation in the compute dtype fp16: W^ = fp16(fl32(v[code] * absmax)).
-* R14 product: out = fp16(X . W^T), evaluated in float64 with one rounding.
+* R13 dequantisation op (the weight handed back in fp16): W^ = fp16(fl32(v[code] * absmax)).
+* R14 product: out[t, n] = fp16(sum_k X[t, k] * v[code[n, k]] * absmax[n, k / 64]),
+      evaluated in float64 with one rounding: the dequantised weight enters the
+      product exactly (the compute dtype of the page concerns how a library
+      evaluates it; any evaluation in fp32 or wider is within the bound the tests
+      derive).
       (Double quantisation of the scales is a storage option of the page, not
       part of this product, and is not built.)
 """
@@ -93,10 +97,17 @@ def dequant_nf4(packed, absmax) -> np.ndarray:
     return prod.reshape(N, K).astype(np.float16)
 
 
+def nf4_weight_exact(packed, absmax) -> np.ndarray:
+    """v[code] * absmax in float64 (exact: a product of two fp32 values), [N, K]."""
+    codes = unpack_codes(packed)
+    N, K = codes.shape
+    v = nf4_levels().astype(np.float64)[codes].reshape(N, K // BLOCK, BLOCK)
+    return (v * np.asarray(absmax, np.float32).astype(np.float64)[..., None]).reshape(N, K)
+
+
 def nf4_gemv(X, packed, absmax) -> np.ndarray:
-    """out = fp16(X . W^T) in float64 with one rounding (reading R14): X fp16 [M, K]."""
+    """out = fp16(X . (v * absmax)^T) in float64 with one rounding (reading R14): X fp16 [M, K]."""
     X = np.asarray(X)
     if X.dtype != np.float16:
         raise TypeError("fp16 X expected")
-    W = dequant_nf4(packed, absmax).astype(np.float64)
-    return (X.astype(np.float64) @ W.T).astype(np.float16)
+    return (X.astype(np.float64) @ nf4_weight_exact(packed, absmax).T).astype(np.float16)
