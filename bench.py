@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--no-other", action="store_true", help="skip the single-linear, OPT MLP and outlier sweep")
     ap.add_argument("--no-shared", action="store_true", help="skip the shared-input layer step")
     ap.add_argument("--no-quant", action="store_true", help="skip the quantiser roofline")
+    ap.add_argument("--no-nf4", action="store_true", help="skip the NF4 decode product")
     ap.add_argument("--cpu-rows", type=int, default=256, help="rows per linear in the CPU oracle sample")
     return ap.parse_args()
 
@@ -303,6 +304,40 @@ def measure_quant(i8, torch, dev, st, world, dist, reps: int = 40):
             "timing": f"CUDA events over {reps} back-to-back calls, inputs rotated over > 2 x L2",
             "kernel_us": "threshold 0: the quantiser kernel alone; op_tau6: memset + quantiser + column zeroing",
             "points": res}
+
+
+def measure_nf4(i8, torch, dev, st, world, dist, reps: int = 20):
+    """The 4-bit NF4 weight-only decode product on the Llama-70B FFN shapes at 1, 4 and 8 tokens:
+    the packed weight (N*K/2 bytes) and its block scales (N*K/16 bytes) stream from HBM every call
+    (117 MB + 15 MB, > L2).  Weights quantised once on the GPU (load time)."""
+    hbm = (measured_peaks() or {}).get("hbm_gbs", 6650.0)
+    points = []
+    for N, K in ((28672, 8192), (8192, 28672)):
+        packed, absmax = i8.i8_nf4_quantize(torch.from_numpy(wl.weight(950 + N, N, K)).to(dev))
+        for M in (1, 4, 8):
+            X, _ = wl.activation(wl.BASE_SEED + 951 + M, M, K, 8, (30.0, 30.0))
+            dX = torch.from_numpy(X).to(dev)
+            out = torch.empty((M, N), dtype=torch.float16, device=dev)
+            for _ in range(3):
+                i8.i8_nf4_gemv(dX, packed, absmax, out=out)
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for _ in range(reps):
+                i8.i8_nf4_gemv(dX, packed, absmax, out=out)
+            e1.record(st)
+            torch.cuda.synchronize(dev)
+            us = e0.elapsed_time(e1) / reps * 1e3
+            byts = N * K // 2 + N * (K // 64) * 4 + 2 * M * K + 2 * M * N
+            gbs = byts / us / 1e3
+            points.append({"shape": f"{M}x{K}->{N}", "tokens": M, "us": round(us, 2), "GB/s": round(gbs, 1),
+                           "frac": round(gbs / hbm, 4)})
+        del packed, absmax
+    return {"kernel": "k_nf4_gemv", "peak_gbs": hbm,
+            "peak_source": "of measured hbm_gbs" if measured_peaks() else "of fallback",
+            "bytes": "N*K/2 + 4*N*K/64 + 2MK + 2MN per call", "points": points}
 
 
 def cpu_per_config(layers_by_key, rows: int, min_seconds: float):
@@ -774,6 +809,11 @@ def run_ours(args):
     if not args.no_quant:
         quant = measure_quant(i8, torch, dev, st, world, dist)
 
+    # ---- the NF4 weight-only decode product (HBM roofline)
+    nf4 = None
+    if not args.no_nf4:
+        nf4 = measure_nf4(i8, torch, dev, st, world, dist)
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -859,11 +899,16 @@ def run_ours(args):
                          "peak_gbs": decode["peak_gbs"],
                          "points": [[q["tokens"], q["outlier_cols"], q["shape"], q["us"], q["GB/s"], q["frac"]]
                                     for q in decode["points"]],
-                         "columns": ["tokens", "outlier_cols", "shape", "us", "GB/s", "frac"]}},
+                         "columns": ["tokens", "outlier_cols", "shape", "us", "GB/s", "frac"]},
+                     "nf4": None if nf4 is None else {
+                         "kernel": nf4["kernel"], "bytes": nf4["bytes"], "peak_gbs": nf4["peak_gbs"],
+                         "points": [[q["shape"], q["us"], q["GB/s"], q["frac"]] for q in nf4["points"]],
+                         "columns": ["shape", "us", "GB/s", "frac"]}},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "decode": decode,
         "quant": quant,
+        "nf4": nf4,
         "backward": backward,
         "other_workloads": other_wl,
         "shared_inputs": shared,

@@ -176,6 +176,41 @@ I8_API i8_status i8_gather_column_blocks(const i8_half* G, int P, int M, int Np,
                                          i8_stream_t stream);
 
 /*
+ * 4-bit NF4 weight-only product, blocksize 64 ("Loading an LLM in 4 bits using
+ * bitsandbytes", sections "Normalized Float" and "Double Quantization": the
+ * nf4 values are optimised for normally distributed weights; weights are
+ * quantised in blocks of 64, each with a 32-bit scale; the product is computed
+ * after dequantisation).  The page prints neither the values nor the rounding
+ * rule; this library takes:
+ *   levels  the NormalFloat construction: with Q the standard normal quantile
+ *           and p* = 1 - (1/32 + 1/30)/2, Q(1/2 + i(p* - 1/2)/8)/Q(p*) for
+ *           i = 1..8, -Q(1/2 + i(p* - 1/2)/7)/Q(p*) for i = 1..7, and 0, as
+ *           fp32, ascending (code 7 is 0, codes 0 and 15 are -1 and +1);
+ *   codes   per block of 64 consecutive weights of a row (K % 64 == 0):
+ *           a = max |w| (fp32), y = fl32(w / a) (0 if a == 0), code = the number
+ *           of midpoints fl32((v_i + v_{i+1})/2) below y (nearest level, ties to
+ *           the lower); byte j of a row holds element 2j in its low nibble and
+ *           element 2j + 1 in its high nibble;
+ *   dequant W^ = fp16(fl32(v[code] * a)).
+ *
+ * i8_nf4_levels — the 16 levels (host memory, 16 floats).  Host only: needs no
+ *   device and is safe to call anywhere.
+ * i8_nf4_quantize — W [N, K] fp16 -> packed [N, K/2] uint8, absmax [N, K/64] fp32.
+ * i8_nf4_dequant — packed, absmax -> W^ [N, K] fp16.
+ * i8_nf4_gemv — the decode product out [M, N] fp16 =
+ *   fp16(sum_k X[t, k] * v[code[n, k]] * absmax[n, k/64]), 1 <= M <= 8 tokens,
+ *   evaluated in fp32 (the block scale applied once per 32 weights).  X [M, K]
+ *   fp16 16-byte aligned; packed 16-byte aligned; absmax 4-byte aligned.
+ */
+I8_API i8_status i8_nf4_levels(float* levels16);
+I8_API i8_status i8_nf4_quantize(const i8_half* W, int N, int K, uint8_t* packed, float* absmax,
+                                 i8_stream_t stream);
+I8_API i8_status i8_nf4_dequant(const uint8_t* packed, const float* absmax, int N, int K, i8_half* W,
+                                i8_stream_t stream);
+I8_API i8_status i8_nf4_gemv(const i8_half* X, int M, const uint8_t* packed, const float* absmax, int N,
+                             int K, i8_half* out, i8_stream_t stream);
+
+/*
  * i8_linear8bit_backward_input — input gradient of the int8 linear layer:
  *   dX[i, k] = fp16( sum_n dY[i, n] * Wt[k, n] ),  fp32 accumulation,
  * i.e. dX = dY . W^ for y = X . W^T + bias with W^ = Wt^T.  With Wt from

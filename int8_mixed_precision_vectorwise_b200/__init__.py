@@ -24,6 +24,10 @@ from ._binding import (  # noqa: F401
     i8_linear8bit_prepare,
     i8_linear8bit_workspace_layout,
     i8_linear8bit_workspace_size,
+    i8_nf4_dequant,
+    i8_nf4_gemv,
+    i8_nf4_levels,
+    i8_nf4_quantize,
     i8_outlier_columns,
     i8_quantize_rowwise,
     i8_read_status,

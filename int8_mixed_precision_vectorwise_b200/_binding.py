@@ -36,6 +36,7 @@ EXPORTS = (
     "i8_linear8bit_multi_workspace_size", "i8_linear8bit_forward_multi",
     "i8_int8_linear_matmul_workspace_size", "i8_int8_linear_matmul_ws", "i8_linear8bit_workspace_layout",
     "i8_linear8bit_backward_input_status", "i8_gather_column_blocks",
+    "i8_nf4_levels", "i8_nf4_quantize", "i8_nf4_dequant", "i8_nf4_gemv",
 )
 
 
@@ -72,6 +73,10 @@ def _declare(lib):
         "i8_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
         "i8_dequant_transposed": (_I, [_P, _P, _I, _I, _P, _P]),
         "i8_gather_column_blocks": (_I, [_P, _I, _I, _I, _P, _P]),
+        "i8_nf4_levels": (_I, [_P]),
+        "i8_nf4_quantize": (_I, [_P, _I, _I, _P, _P, _P]),
+        "i8_nf4_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
+        "i8_nf4_gemv": (_I, [_P, _I, _P, _P, _I, _I, _P, _P]),
         "i8_linear8bit_backward_input": (_I, [_P, _P, _I, _I, _I, _P, _P]),
         "i8_linear8bit_multi_workspace_size": (_S, [_I, _I, _I, _P, _I]),
         "i8_linear8bit_forward_multi": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _F, _P, _S, _I, _P]),
@@ -291,6 +296,48 @@ def i8_gather_column_blocks(G, out=None):
     out = _out(out, torch.float16, "out", (M, P * Np), G.device)
     _check("i8_gather_column_blocks", lib().i8_gather_column_blocks(
         _ptr(G), P, M, Np, _ptr(out), _stream(G.device)))
+    return out
+
+
+def i8_nf4_levels():
+    """The 16 NF4 levels (host, fp32 list, ascending)."""
+    buf = (ctypes.c_float * 16)()
+    _check("i8_nf4_levels", lib().i8_nf4_levels(buf))
+    return list(buf)
+
+
+def i8_nf4_quantize(W, packed=None, absmax=None):
+    """Blockwise (64) NF4 quantisation of an fp16 weight [N, K]: returns (packed [N, K/2] uint8,
+    absmax [N, K/64] fp32)."""
+    _need(W, torch.float16, "W", 2)
+    N, K = W.shape
+    packed = _out(packed, torch.uint8, "packed", (N, K // 2), W.device)
+    absmax = _out(absmax, torch.float32, "absmax", (N, K // 64), W.device)
+    _check("i8_nf4_quantize", lib().i8_nf4_quantize(_ptr(W), N, K, _ptr(packed), _ptr(absmax), _stream(W.device)))
+    return packed, absmax
+
+
+def i8_nf4_dequant(packed, absmax, W=None):
+    """fp16 [N, K] dequantised NF4 weight."""
+    _need(packed, torch.uint8, "packed", 2)
+    N, H = packed.shape
+    K = 2 * H
+    _arg(absmax, torch.float32, "absmax", (N, K // 64), packed.device)
+    W = _out(W, torch.float16, "W", (N, K), packed.device)
+    _check("i8_nf4_dequant", lib().i8_nf4_dequant(_ptr(packed), _ptr(absmax), N, K, _ptr(W), _stream(packed.device)))
+    return W
+
+
+def i8_nf4_gemv(X, packed, absmax, out=None):
+    """out [M, N] = fp16(X [M, K] . NF4 weight^T), 1 <= M <= 8."""
+    _need(X, torch.float16, "X", 2)
+    M, K = X.shape
+    dev = X.device
+    _arg(packed, torch.uint8, "packed", (packed.shape[0], K // 2), dev)
+    N = packed.shape[0]
+    _arg(absmax, torch.float32, "absmax", (N, K // 64), dev)
+    out = _out(out, torch.float16, "out", (M, N), dev)
+    _check("i8_nf4_gemv", lib().i8_nf4_gemv(_ptr(X), M, _ptr(packed), _ptr(absmax), N, K, _ptr(out), _stream(dev)))
     return out
 
 

@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libi8lt.so")
-SOURCES = ["i8lt_api.cu", "quant_kernels.cu", "decode_prep.cu", "gemm_tcgen05.cu", "gemm_decode.cu", "linear_small.cu"]
+SOURCES = ["i8lt_api.cu", "quant_kernels.cu", "decode_prep.cu", "gemm_tcgen05.cu", "gemm_decode.cu", "linear_small.cu", "nf4.cu"]
 HEADERS = ["ptx.cuh", "kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

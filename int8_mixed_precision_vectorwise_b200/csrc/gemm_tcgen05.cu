@@ -45,6 +45,7 @@
 #include <cuda_fp16.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -358,6 +359,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint8_t* stg = smem + STG_OFF + ew * 2 * STG_BYTES;
     int stg_i = 0;
     int it = 0;
+    auto run_units = [&](auto defer_tag) {
+    constexpr bool DEFER = decltype(defer_tag)::value;  // the value of `defer`, as a constant
     for (int u = pair; u < U.units; u += npairs, ++it) {  // abort is seen by the wait below
       int tile, half;
       U.at(u, tile, half);
@@ -380,7 +383,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = row_base + g + 8 * i;
-        sa4[i] = (!RAW && !F16 && r < M) ? __ldg(p.SCA + r) * (defer ? (1.0f / 127.0f) : (1.0f / 16129.0f)) : 0.f;
+        sa4[i] = (!RAW && !F16 && r < M) ? __ldg(p.SCA + r) * (DEFER ? (1.0f / 127.0f) : (1.0f / 16129.0f)) : 0.f;
       }
       // Few outliers: the A fragments (X[:, O] rows) of the 16-wide outlier
       // product.  The gathered operands store each group of 16 outlier columns
@@ -434,7 +437,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       tc_fence_after_sync();
       const uint32_t t_int = tmem_base + lane_off + static_cast<uint32_t>(buf * BN + col_off);
-      if (defer) {
+      if constexpr (DEFER) {
         // Many outlier columns, phase 1: the int32 accumulator becomes fp32
         // C * SCA / 127 in place; the MMA thread then adds the outlier product
         // onto it (fragment element e of row block rb is row rb*16 + g + 8*((e >> 1) & 1)).
@@ -473,14 +476,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         if (cc + 1 < nch) fetch_chunk(cc + 1);
         uint32_t c[2][16];  // int32 accumulators of row blocks 0 / 1
-        if (!F16 && !defer) {
+        if (!F16 && !DEFER) {
           tmem_ld_16x256b_x4(t_int + cc * 32, c[0]);
           tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, c[1]);
         }
         // fp32 accumulators: C * SCA / 127 plus the outlier product (many-outlier
         // path) or, in the fp16 mode, the whole product
         uint32_t f[2][16];
-        if (F16 || defer) {
+        if (F16 || DEFER) {
           tmem_ld_16x256b_x4(t_int + cc * 32, f[0]);
           tmem_ld_16x256b_x4(t_int + (16u << 16) + cc * 32, f[1]);
         }
@@ -523,7 +526,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             if (small_o) {
               mma_16x8x16_f16(d, af[rb], bf_c[cb][0], bf_c[cb][1]);
-            } else if (F16 || defer) {
+            } else if (F16 || DEFER) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) d[e] = __uint_as_float(f[rb][4 * cb + e]);
             }
@@ -531,7 +534,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             for (int hh = 0; hh < 2; ++hh) {
               if constexpr (F16) {
                 halves[rb][cb][hh] = pack_half2(d[2 * hh], d[2 * hh + 1]);
-              } else if (defer) {
+              } else if constexpr (DEFER) {
                 // (C * SCA / 127 + outlier product) * SCB / 127 + bias
                 halves[rb][cb][hh] = pack_half2(fmaf(d[2 * hh], sb0 * (1.0f / 127.0f), b0),
                                                 fmaf(d[2 * hh + 1], sb1 * (1.0f / 127.0f), b1));
@@ -595,6 +598,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0_leader + static_cast<uint32_t>(buf) * 8u);
     }
+    };
+    // one instruction stream per way of adding many outlier columns, so the
+    // common path carries no per-element test of it
+    if (defer)
+      run_units(std::true_type{});
+    else
+      run_units(std::false_type{});
     if (!RAW && p.tma_store && lane == 0) tma_store_wait_all<0>();
     __syncwarp();
   }

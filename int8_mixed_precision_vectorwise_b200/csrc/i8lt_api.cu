@@ -219,9 +219,15 @@ i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, in
 // Few-token GEMM: 128-byte K boxes per pipeline stage (512 bytes of each
 // weight row per stage) and the grid of the stream-K split (one CTA per SM, at
 // most kDecodeMaxGrid, never more CTAs than (tile, stage) work items).
+// `prep_elems` is the M*K the preparation kernel before it quantises: when it
+// is large, that kernel's cluster keeps its SMs busy for several microseconds
+// while the GEMM's CTAs would wait for them with an equal share of the weight
+// stream, so the GEMM leaves those SMs out.
 constexpr int kDecodeBoxes = 4;
-int decode_grid(int N, int K, int sms) {
+constexpr long long kDecodeHeavyPrep = 16LL * 16384;
+int decode_grid(int N, int K, int sms, long long prep_elems) {
   const int total = ((N + 127) / 128) * ((K + 128 * kDecodeBoxes - 1) / (128 * kDecodeBoxes));
+  if (prep_elems >= kDecodeHeavyPrep) sms -= i8lt::kDecodePrepCluster;
   int grid = sms < i8lt::kDecodeMaxGrid ? sms : i8lt::kDecodeMaxGrid;
   return grid > total ? total : grid;
 }
@@ -294,8 +300,7 @@ i8_status enqueue_prepare(const i8_half* X, const int8_t* CB, int M, int N, int 
   }
   // status word, counts and bitmap are contiguous: one memset clears them
   if (cudaMemsetAsync(workspace, 0, L.clear_bytes, st) != cudaSuccess) return I8_ERR_CUDA;
-  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr,
-                                                    sms, w.hdr, kWaitLimitNs, st));
+  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, w.CA, w.SCA, outliers ? w.bitmap : nullptr, st));
   if (s != I8_OK || !outliers) return s;
   return cuda_status(i8lt::launch_outlier_prepare(w.bitmap, K, cap, reinterpret_cast<int32_t*>(w.hdr + 2),
                                                   reinterpret_cast<int32_t*>(w.hdr + 1), w.idx, w.hdr, w.CA, Xh, M,
@@ -334,7 +339,8 @@ i8_status enqueue_gemm(const int8_t* CB, const float* SCB, const i8_half* bias, 
       return I8_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return I8_ERR_CUDA;
-    return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms), kDecodeBoxes, true, st));
+    return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms, static_cast<long long>(M) * K),
+                                                kDecodeBoxes, true, st));
   }
   GemmArgs a{};
   a.M = M;
@@ -486,8 +492,7 @@ i8_status i8_quantize_rowwise(const i8_half* X, int M, int K, float threshold, i
   }
   const int sms = num_sms();
   if (sms <= 0) return I8_ERR_CUDA;
-  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, threshold > 0.f ? bitmap : nullptr,
-                                                    sms, nullptr, kWaitLimitNs, st));
+  i8_status s = cuda_status(i8lt::launch_quant_rows(Xh, M, K, threshold, CA, SCA, threshold > 0.f ? bitmap : nullptr, st));
   if (s != I8_OK || threshold == 0.f) return s;
   return cuda_status(i8lt::launch_zero_outlier_cols(bitmap, M, K, CA, sms, st));
 }
@@ -567,8 +572,9 @@ i8_status i8_int8_linear_matmul_ws(const int8_t* A, const int8_t* B, int M, int 
   if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, 128, 128) ||
       !encode_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, M, K, 128, i8lt::kDecodeMaxTokens))
     return I8_ERR_CUDA;
-  // no programmatic overlap: B may be written by the work queued just before
-  return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms), kDecodeBoxes, false, st));
+  // no programmatic overlap: B may be written by the work queued just before;
+  // no preparation kernel runs beside it
+  return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms, 0), kDecodeBoxes, false, st));
 }
 
 i8_status i8_linear8bit_workspace_layout(int M, int N, int K, int max_outlier_cols, i8_workspace_layout* layout) {
@@ -621,6 +627,52 @@ i8_status i8_dequant_transposed(const int8_t* CB, const float* SCB, int N, int K
   if (!aligned16(CB) || !aligned16(Wt)) return I8_ERR_UNSUPPORTED_SHAPE;
   return cuda_status(i8lt::launch_dequant_t(CB, SCB, N, K, reinterpret_cast<__half*>(Wt),
                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_nf4_levels(float* levels16) {
+  if (!levels16) return I8_ERR_INVALID_ARG;
+  const i8lt::Nf4Tables t = i8lt::nf4_tables();
+  for (int i = 0; i < 16; ++i) levels16[i] = t.level[i];
+  return I8_OK;
+}
+
+i8_status i8_nf4_quantize(const i8_half* W, int N, int K, uint8_t* packed, float* absmax, i8_stream_t stream) {
+  if (!W || !packed || !absmax) return I8_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (K % 64 != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || (reinterpret_cast<uintptr_t>(absmax) & 3u) != 0)
+    return I8_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_nf4_quantize(reinterpret_cast<const __half*>(W), N, K, packed, absmax, sms,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_nf4_dequant(const uint8_t* packed, const float* absmax, int N, int K, i8_half* W, i8_stream_t stream) {
+  if (!W || !packed || !absmax) return I8_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (K % 64 != 0) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(packed) || (reinterpret_cast<uintptr_t>(absmax) & 3u) != 0)
+    return I8_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_nf4_dequant(packed, absmax, N, K, reinterpret_cast<__half*>(W), sms,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+i8_status i8_nf4_gemv(const i8_half* X, int M, const uint8_t* packed, const float* absmax, int N, int K, i8_half* out,
+                      i8_stream_t stream) {
+  if (!X || !packed || !absmax || !out) return I8_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return I8_ERR_INVALID_ARG;
+  if (K % 64 != 0 || M > i8lt::kNf4MaxTokens) return I8_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(packed) || (reinterpret_cast<uintptr_t>(absmax) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(out) & 1u) != 0)
+    return I8_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
+  return cuda_status(i8lt::launch_nf4_gemv(reinterpret_cast<const __half*>(X), M, packed, absmax, N, K,
+                                           reinterpret_cast<__half*>(out), sms,
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 i8_status i8_gather_column_blocks(const i8_half* G, int P, int M, int Np, i8_half* out, i8_stream_t stream) {

@@ -9,10 +9,9 @@
 
 namespace i8lt {
 
-// bitmap: zeroed outlier bitmap to OR into (required when tau > 0).  status
-// (nullable): device word that a pipeline-wait timeout of the ring kernel sets.
+// bitmap: zeroed outlier bitmap to OR into (required when tau > 0).
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
-                              int num_sms, uint32_t* status, uint64_t limit_ns, cudaStream_t st);
+                              cudaStream_t st);
 cudaError_t launch_zero_outlier_cols(const uint32_t* bitmap, int M, int K, int8_t* CA, int num_sms,
                                      cudaStream_t st);
 cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32_t* total_out, int32_t* used_out,
@@ -137,6 +136,24 @@ size_t linear_small_smem(int K);
 cudaError_t launch_linear_small(const CUtensorMap& tmW, const __half* X, int M, int N, int K, float tau, int cap,
                                 const float* SCB, const __half* bias, __half* out, uint32_t* hdr, uint64_t limit_ns,
                                 bool reset_status, cudaStream_t st);
+
+// 4-bit NF4 weight-only product, blocksize 64.  Nf4Tables holds the 16 levels
+// (ascending, level[7] = 0) and the 15 midpoints between neighbours (fp32),
+// computed on the host; passed to the kernels by value.
+struct Nf4Tables {
+  float level[16];
+  float mid[16];
+};
+constexpr int kNf4MaxTokens = 8;
+Nf4Tables nf4_tables();
+// W [N, K] fp16 -> packed [N, K/2] (element 2j low nibble of byte j), absmax [N, K/64]; K % 64 == 0.
+cudaError_t launch_nf4_quantize(const __half* W, int N, int K, uint8_t* packed, float* absmax, int num_sms,
+                                cudaStream_t st);
+cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int N, int K, __half* W, int num_sms,
+                               cudaStream_t st);
+// out [M, N] fp16 = X [M, K] . dequantised weight^T, 1 <= M <= kNf4MaxTokens.
+cudaError_t launch_nf4_gemv(const __half* X, int M, const uint8_t* packed, const float* absmax, int N, int K,
+                            __half* out, int num_sms, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 

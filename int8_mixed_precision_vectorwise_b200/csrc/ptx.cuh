@@ -117,27 +117,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
       : "memory");
 }
 
-// Barrier `id` (1..15) over `nthreads` threads of the CTA (a multiple of 32);
-// lets a subset of the warps synchronise without the others.
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// The same barrier, also returning whether `pred` was true in any of the
-// participating threads (one uniform answer for all of them).
-__device__ __forceinline__ bool named_bar_any(uint32_t id, uint32_t nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, %2, %3, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 // ------------------------------------------------------------------ tcgen05
 // TMEM allocation: executed by one full warp; writes the TMEM base address to
 // shared memory.

@@ -11,7 +11,6 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
-#include <atomic>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -167,100 +166,6 @@ __global__ void __launch_bounds__(256, (VPT > 8 ? 1 : 5)) k_quant_rows(const __h
     __syncthreads();
     sbm_flush(sbm, nwords, bitmap);
   }
-}
-
-// Persistent ring quantiser for rows of 2 KB .. 32 KB (1024 <= K <= 16384).
-// Each CTA (one per SM) owns a contiguous range of rows.  Lane 0 of warp 0
-// streams whole rows of X into a ring of shared-memory slots with 1-D bulk
-// copies, so up to `slots` rows (~200 KB) per SM are in flight while rows are
-// being quantised; a slot is refilled as soon as the row in it is done.  Each
-// of the other `nwc` warps quantises its own rows (row j of the range goes to
-// warp j % nwc) from shared memory, with warp-level reductions only, so many
-// rows are in progress at once.  `slots` is a multiple of `nwc`, so a slot
-// only ever holds rows of one warp, which takes them in order: no wait can
-// run a whole phase ahead of the slot's barrier.  Per row: absmax over the row (elements at or above the
-// threshold left out and marked in the CTA's outlier bitmap), one fp32
-// division, codes written with 8-byte coalesced stores.  Every wait is
-// bounded; a timeout sets *status (when given), the warps leave their loops
-// and the producer first waits, bounded, for its copies.
-constexpr int kRingWarps = 8;        // most consumer warps, one row each at a time
-constexpr int kRingThreads = 32 * (1 + kRingWarps);
-constexpr int kRingMaxSlots = 32;
-constexpr int kRingSlotBudget = 200 * 1024;
-
-__global__ void __launch_bounds__(kRingThreads, 1)
-    k_quant_rows_ring(const __half* __restrict__ X, int M, int K, float tau, int8_t* __restrict__ CA,
-                      float* __restrict__ SCA, uint32_t* __restrict__ bitmap, int rows_per_cta, int slots,
-                      int nwc, uint32_t* status, uint64_t limit_ns) {
-  extern __shared__ __align__(128) uint8_t rsm[];
-  const int row_bytes = 2 * K;
-  uint8_t* ring = rsm;
-  uint64_t* full = reinterpret_cast<uint64_t*>(rsm + static_cast<size_t>(slots) * row_bytes);
-  uint64_t* empty = full + slots;
-  volatile int* s_abort = reinterpret_cast<volatile int*>(empty + slots);
-  uint32_t* sbm = reinterpret_cast<uint32_t*>(empty + slots) + 4;
-  pdl_launch_dependents();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = blockIdx.x * rows_per_cta;
-  const int n = max(0, min(rows_per_cta, M - r0));
-  const int nvec = K >> 3, nwords = (K + 31) >> 5;
-  const bool use_tau = tau > 0.f;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < slots; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);  // the warp that quantised the slot's row
-    }
-    *s_abort = 0;
-    fence_barrier_init();
-  }
-  if (use_tau) sbm_clear(sbm, nwords);
-  __syncthreads();
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      uint32_t filled = 0, fill_parity = 0;
-      for (int j = 0; j < n; ++j) {
-        const int s = j % slots;
-        const uint32_t use = static_cast<uint32_t>(j / slots);
-        if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1u, s_abort, status, limit_ns)) break;
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(row_bytes));
-        filled |= 1u << s;
-        fill_parity = (fill_parity & ~(1u << s)) | ((use & 1u) << s);
-        bulk_load(ring + static_cast<size_t>(s) * row_bytes, X + static_cast<size_t>(r0 + j) * K,
-                  static_cast<uint32_t>(row_bytes), &full[s]);
-      }
-      if (*s_abort) {  // never leave while a copy may still be landing in shared memory
-        int never = 0;
-        for (int s = 0; s < slots; ++s)
-          if (filled & (1u << s)) mbar_wait_bounded(&full[s], (fill_parity >> s) & 1u, &never, nullptr, limit_ns);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ---------------------------------------------------------------- consumers
-    for (int j = warp - 1; warp <= nwc && j < n; j += nwc) {
-      const int s = j % slots;
-      int ok = 0;
-      if (lane == 0) ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / slots) & 1u, s_abort, status, limit_ns);
-      if (!__shfl_sync(kFull, ok, 0)) break;
-      const uint4* v = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(s) * row_bytes);
-      float amax = 0.f;
-#pragma unroll 4
-      for (int vi = lane; vi < nvec; vi += 32) fold8(v[vi], vi, tau, use_tau, amax, sbm);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-      const float r = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
-      const int row = r0 + j;
-      if (lane == 0) SCA[row] = amax;
-      uint2* cr = reinterpret_cast<uint2*>(CA + static_cast<size_t>(row) * K);
-#pragma unroll 4
-      for (int vi = lane; vi < nvec; vi += 32) cr[vi] = quant8(v[vi], r);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);  // the slot may be refilled
-    }
-  }
-  __syncthreads();
-  if (use_tau) sbm_flush(sbm, nwords, bitmap);
 }
 
 // Rows too long to cache in registers: one block per row, X read twice (the
@@ -574,33 +479,9 @@ cudaError_t launch_gather_column_blocks(const __half* G, int P, int M, int Np, _
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_quant_rows(const __half* X, int M, int K, float tau, int8_t* CA, float* SCA, uint32_t* bitmap,
-                              int num_sms, uint32_t* status, uint64_t limit_ns, cudaStream_t st) {
+                              cudaStream_t st) {
   const size_t smem = tau > 0.f ? static_cast<size_t>((K + 31) / 32) * 4 : 0;
   const int nvec = K / 8;
-  if (K >= 1024 && K <= 16384 && num_sms > 0) {
-    // rows of 2 KB .. 32 KB: the persistent ring kernel, one CTA per SM
-    const int row_bytes = 2 * K;
-    // consumer warps, and slots rounded down to a multiple of them (each warp its own slots)
-    const int nwc = std::min(kRingWarps, std::min(kRingMaxSlots, kRingSlotBudget / row_bytes));
-    const int slots = (std::min(kRingMaxSlots, kRingSlotBudget / row_bytes) / nwc) * nwc;
-    const size_t ring_smem = static_cast<size_t>(slots) * row_bytes + static_cast<size_t>(slots) * 16 + 16 +
-                             static_cast<size_t>((K + 31) / 32) * 4;
-    static std::atomic<bool> attr_done[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-    if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
-      cudaError_t e = cudaFuncSetAttribute(k_quant_rows_ring, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kRingSlotBudget + 8 * 1024);
-      if (e != cudaSuccess) return e;
-      if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
-    }
-    int grid = std::min(M, num_sms);
-    const int rows_per_cta = (M + grid - 1) / grid;
-    grid = (M + rows_per_cta - 1) / rows_per_cta;
-    k_quant_rows_ring<<<grid, kRingThreads, ring_smem, st>>>(X, M, K, tau, CA, SCA, bitmap, rows_per_cta, slots,
-                                                              nwc, status, limit_ns);
-    return cudaGetLastError();
-  }
   // One row per group of threads with the row in registers (one pass over X),
   // grids of many small blocks so that enough rows are in flight per SM; rows
   // beyond 32768 columns stream twice.
@@ -631,11 +512,15 @@ cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32
                                    int32_t* idx_out, uint32_t* status, int8_t* CA, const __half* X, int M,
                                    __half* XO, const int8_t* CB, int N, __half* WO, int ld_o, int num_sms,
                                    cudaStream_t st) {
-  // work items: (row, 16-position group); a grid of up to 8 blocks per SM
+  // work items: (row, 16-position group), at most as many as the capacity
+  // allows.  The grid is capped at 2 blocks per SM: the kernel is launched as a
+  // programmatic dependent of the quantiser, so its blocks can become resident
+  // while the quantiser still runs and would take warp slots from it; the
+  // item loop strides over the grid.
   const int rows = ((XO || CA) ? M : 0) + (WO ? N : 0);
   const int groups = cap <= 16 ? 1 : ((cap + 63) / 64) * 4;
   const long long items = static_cast<long long>(rows) * groups;
-  const int blocks = static_cast<int>(std::max<long long>(1, std::min<long long>((items + 255) / 256, num_sms * 8LL)));
+  const int blocks = static_cast<int>(std::max<long long>(1, std::min<long long>((items + 255) / 256, num_sms * 2LL)));
   const size_t smem = static_cast<size_t>(max(cap, 1)) * sizeof(int32_t);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks, 1, 1);

@@ -244,3 +244,23 @@ def test_int8_rounding_by_added_constant_is_round_half_even():
     low = (s.view(np.uint32) & np.uint32(0xFF)).astype(np.uint8).view(np.int8)
     want = np.rint(t.astype(np.float64))                     # numpy rint: half to even
     assert np.array_equal(low.astype(np.int64), ((want.astype(np.int64) + 128) % 256) - 128)
+
+
+def test_nf4_levels_match_oracle_bit_for_bit():
+    """The library computes the NF4 levels on the host with its own inverse normal CDF;
+    they must equal the oracle's (scipy) values as fp32 bit patterns."""
+    import numpy as np
+    from int8_mixed_precision_vectorwise_b200 import _binding as b
+    from oracle import nf4
+    got = np.array(b.i8_nf4_levels(), np.float32)
+    assert np.array_equal(got.view(np.uint32), nf4.nf4_levels().view(np.uint32))
+
+
+def test_nf4_rejects(lib):
+    assert lib.i8_nf4_levels(None) == 1
+    assert lib.i8_nf4_quantize(None, 4, 64, FAKE, FAKE, None) == 1
+    assert lib.i8_nf4_quantize(FAKE, 4, 96, FAKE, FAKE, None) == 2          # K % 64
+    assert lib.i8_nf4_gemv(FAKE, 0, FAKE, FAKE, 4, 64, FAKE, None) == 1
+    assert lib.i8_nf4_gemv(FAKE, 9, FAKE, FAKE, 4, 64, FAKE, None) == 2      # at most 8 tokens
+    assert lib.i8_nf4_gemv(FAKE_MIS, 1, FAKE, FAKE, 4, 64, FAKE, None) == 2
+    assert lib.i8_nf4_dequant(FAKE, FAKE, 4, 100, FAKE, None) == 2
