@@ -16,17 +16,17 @@
 //           (fp32 accumulation, the block scale applied once per half block)
 //
 // The product streams the packed weight once (K/2 bytes per row plus K/16
-// bytes of scales); for few tokens it is bound by HBM and by the unpacking
-// work, so it runs on the CUDA cores: each warp takes 4 rows at a time (four
-// independent 16-byte loads per lane in flight), X is staged in shared memory
-// as fp32 chunks that all warps of the CTA share, and the 16 levels sit in
-// shared memory (16 banks: lanes reading different levels never conflict).
+// bytes of scales).  For few tokens it is bound by HBM and by the unpacking
+// work (a shared-memory level lookup per weight), so it runs on the CUDA
+// cores with packed fp32 FMAs; the layout is described at k_nf4_gemv.
 #include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace i8lt {
 
@@ -35,7 +35,8 @@ namespace {
 constexpr int NB = 64;            // weights per scale block
 constexpr int NF_WARPS = 8;
 constexpr int NF_THREADS = 32 * NF_WARPS;
-constexpr int NF_X_FLOATS = 8192; // fp32 elements of X staged per chunk (32 KB)
+constexpr int NF_XBUF = 4096;     // fp32 elements of X per staging buffer (16 KB, two buffers)
+constexpr int NF_STEP = 256;      // weights of a row per step of an octet (128 bytes)
 
 // Standard normal quantile by Newton's method on Phi(x) = erfc(-x / sqrt 2) / 2.
 double normal_quantile(double p) {
@@ -96,7 +97,9 @@ __global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__
                                                      const float* __restrict__ absmax, int N, int K, Nf4Tables tb,
                                                      __half* __restrict__ W) {
   __shared__ float lut[16];
-  if (threadIdx.x < 16) lut[threadIdx.x] = tb.level[threadIdx.x];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (threadIdx.x == i) lut[i] = tb.level[i];
   __syncthreads();
   const size_t nbytes = static_cast<size_t>(N) * K / 2;
   for (size_t j = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; j < nbytes;
@@ -108,94 +111,216 @@ __global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__
   }
 }
 
-// out [M, N] = fp16(X [M, K] . W^T) with MT >= M token slots (a power of two);
-// each warp works on R rows at once (fewer for more tokens, to stay in registers).
+// out [M, N] = fp16(X [M, K] . W^T), MT >= M token slots (1, 2, 4 or 8).
+//
+// Layout of the work: eight lanes (an octet) share one row and read its 128-byte
+// segment of 256 weights per step, lane q taking the 32 weights k0 + 32q ..
+// k0 + 32q + 31 (one 16-byte load, half a scale block).  A warp's four octets take
+// four consecutive rows, R such groups at a time, so a CTA of 8 warps owns
+// 32R consecutive rows.  The CTA walks its K range (all of K, or 1/S of it
+// when S CTAs of a cluster split K) in chunks of X staged as fp32 in shared
+// memory, double-buffered: the next chunk is loaded into registers while the
+// current one is used and stored behind it, one barrier per chunk.  In a chunk
+// the 16-byte granule g of token row t sits at g ^ ((k >> 5) & 7), so the eight
+// lanes of an octet, which read the same granule offset of eight different
+// 32-weight groups, hit eight different bank groups, and the four octets of a
+// warp read the same addresses (broadcast).  The weight codes of the next step
+// are loaded while the current step is computed.
+//
+// Arithmetic (fp32): per row, token and half block, two chains of 16 fused
+// multiply-adds (even and odd k, one packed f32x2 FMA per pair of k), their sum
+// times the block scale added to the lane's running sum; then a 3-level
+// shuffle sum over the octet and, with S > 1, the S partial sums of the cluster
+// added in rank order through distributed shared memory.  Deterministic.
 template <int MT, int R>
-__global__ void __launch_bounds__(NF_THREADS) k_nf4_gemv(const __half* __restrict__ X, int M,
-                                                         const uint8_t* __restrict__ packed,
-                                                         const float* __restrict__ absmax, int N, int K,
-                                                         Nf4Tables tb, __half* __restrict__ out) {
+struct Nf4Shape {
+  static constexpr int KC = NF_XBUF / MT;          // k per chunk (a multiple of 256)
+  static constexpr int ROWS = 32 * R;              // rows per CTA
+  static constexpr int STEPS = KC / NF_STEP;       // 256-weight steps per chunk
+};
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float lut_at(const float* lut, uint32_t byte_off) {
+  return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(lut) + byte_off);
+}
+
+template <int MT, int R>
+__global__ void __launch_bounds__(NF_THREADS, (MT <= 2 && R <= 2) ? 3 : 2) k_nf4_gemv(const __half* __restrict__ X, int M,
+                                                            const uint8_t* __restrict__ packed,
+                                                            const float* __restrict__ absmax, int N, int K,
+                                                            Nf4Tables tb, int S, __half* __restrict__ out) {
+  using Sh = Nf4Shape<MT, R>;
   __shared__ float lut[16];
-  __shared__ __align__(16) float xs[NF_X_FLOATS];  // [MT][kc] chunk of X as fp32
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x < 16) lut[threadIdx.x] = tb.level[threadIdx.x];
-  const int kc_max = NF_X_FLOATS / MT;             // a multiple of 512 (MT <= 16)
-  const int rows_cta = NF_WARPS * R;
+  __shared__ __align__(16) float xs[2][NF_XBUF];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int oct = lane >> 3, q = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)                     // constant indices keep the tables in the parameter space
+    if (tid == i) lut[i] = tb.level[i];
+
+  // this CTA's rows and K range (S CTAs of one cluster share the rows)
+  const int split = S > 1 ? static_cast<int>(blockIdx.x % S) : 0;
+  const int rb = S > 1 ? static_cast<int>(blockIdx.x / S) : static_cast<int>(blockIdx.x);
+  const int nsteps = (K + NF_STEP - 1) / NF_STEP;
+  const int s0 = static_cast<int>(static_cast<long long>(split) * nsteps / S);
+  const int s1 = static_cast<int>(static_cast<long long>(split + 1) * nsteps / S);
+  const int kb = s0 * NF_STEP, ke = min(K, s1 * NF_STEP);
+  const int T = s1 - s0;                           // steps of this CTA
+  const int nchunks = (T + Sh::STEPS - 1) / Sh::STEPS;
   const size_t row_bytes = static_cast<size_t>(K) / 2;
   const int blocks_row = K / NB;
-  for (int g = blockIdx.x; g * rows_cta < N; g += gridDim.x) {
-    const int n0 = g * rows_cta + warp * R;        // this warp's rows n0 .. n0 + R - 1
-    float acc[R][MT];
+  int rows[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+  for (int i = 0; i < R; ++i) rows[i] = rb * Sh::ROWS + (warp * R + i) * 4 + oct;
+
+  // weight codes and block scales of step st for this lane's R rows (zero past the range)
+  auto load_step = [&](int st, uint4 (&qv)[R], float (&av)[R]) {
+    const int kg = kb + st * NF_STEP + 32 * q;
+    const bool ok = kg < ke;
 #pragma unroll
-      for (int t = 0; t < MT; ++t) acc[r][t] = 0.f;
-    for (int k0 = 0; k0 < K; k0 += kc_max) {
-      const int kc = min(kc_max, K - k0);          // a multiple of 64
-      __syncthreads();                             // the previous chunk is no longer read
-      for (int i = threadIdx.x; i < MT * (kc / 2); i += NF_THREADS) {
-        const int t = i / (kc / 2), j = i - t * (kc / 2);
-        float2 f = make_float2(0.f, 0.f);
-        if (t < M) f = __half22float2(*reinterpret_cast<const __half2*>(X + static_cast<size_t>(t) * K + k0 + 2 * j));
-        *reinterpret_cast<float2*>(xs + t * kc + 2 * j) = f;
-      }
-      __syncthreads();
-      // a lane takes 32 consecutive weights (16 bytes, half a scale block) per row and step
-      const int units = kc / 32;
-      for (int u0 = 0; u0 < units; u0 += 32) {
-        const int u = u0 + lane;
-        if (u >= units) continue;
-        const int kk = 32 * u;                     // offset in the chunk
-        uint4 q[R];
-        float a[R];
+    for (int i = 0; i < R; ++i) {
+      const size_t n = static_cast<size_t>(min(rows[i], N - 1));  // rows past N repeat the last; never stored
+      qv[i] = ok ? __ldcs(reinterpret_cast<const uint4*>(packed + n * row_bytes + kg / 2)) : make_uint4(0, 0, 0, 0);
+      av[i] = ok ? __ldg(absmax + n * blocks_row + kg / NB) : 0.f;
+    }
+  };
+  // X chunk c as fp16 pairs in registers (8 per thread), zero past M or the range
+  constexpr int XPT = NF_XBUF / 2 / NF_THREADS;
+  uint32_t xr[XPT];
+  auto load_chunk = [&](int c) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const int n = min(n0 + r, N - 1);        // rows past N repeat the last one; never stored
-          q[r] = __ldcs(reinterpret_cast<const uint4*>(packed + static_cast<size_t>(n) * row_bytes + (k0 + kk) / 2));
-          a[r] = __ldg(absmax + static_cast<size_t>(n) * blocks_row + (k0 + kk) / NB);
+    for (int j = 0; j < XPT; ++j) {
+      const int p = tid + NF_THREADS * j;
+      const int t = p / (Sh::KC / 2), kp = p % (Sh::KC / 2);
+      const int kg = kb + c * Sh::KC + 2 * kp;
+      xr[j] = (t < M && kg < ke) ? __ldg(reinterpret_cast<const uint32_t*>(X + static_cast<size_t>(t) * K + kg)) : 0u;
+    }
+  };
+  auto store_chunk = [&](float* buf) {
+#pragma unroll
+    for (int j = 0; j < XPT; ++j) {
+      const int p = tid + NF_THREADS * j;
+      const int t = p / (Sh::KC / 2), kp = p % (Sh::KC / 2);
+      const int fi = t * Sh::KC + 2 * kp;
+      const int phys = (fi >> 2) ^ ((kp >> 4) & 7);
+      __half2 h;
+      memcpy(&h, &xr[j], 4);
+      *reinterpret_cast<float2*>(buf + 4 * phys + (fi & 3)) = __half22float2(h);
+    }
+  };
+
+  float acc[R][MT];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int t = 0; t < MT; ++t) acc[i][t] = 0.f;
+
+  uint4 qn[R];
+  float an[R];
+  if (T > 0) load_step(0, qn, an);
+  load_chunk(0);
+  store_chunk(xs[0]);
+  __syncthreads();
+  for (int c = 0; c < nchunks; ++c) {
+    if (c + 1 < nchunks) load_chunk(c + 1);
+    const float* xb = xs[c & 1];
+    for (int j = 0; j < Sh::STEPS; ++j) {
+      const int st = c * Sh::STEPS + j;
+      if (st >= T) break;
+      uint4 qc[R];
+      float ac[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) { qc[i] = qn[i]; ac[i] = an[i]; }
+      if (st + 1 < T) load_step(st + 1, qn, an);
+      float2 s[R][MT];
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int t = 0; t < MT; ++t) s[i][t] = make_float2(0.f, 0.f);
+      const int g0 = (NF_STEP * j + 32 * q) >> 2;  // granule of this lane's first weight (token 0)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t eb[R], ob[R];                     // byte j: 4 x code of weight 8w + 2j (eb) and 8w + 2j + 1 (ob)
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+          const uint32_t wd = w == 0 ? qc[i].x : (w == 1 ? qc[i].y : (w == 2 ? qc[i].z : qc[i].w));
+          eb[i] = (wd << 2) & 0x3C3C3C3Cu;
+          ob[i] = (wd >> 2) & 0x3C3C3C3Cu;
         }
-        float s[R][MT];
 #pragma unroll
-        for (int r = 0; r < R; ++r)
+        for (int h = 0; h < 2; ++h) {
+          float4 xv[MT];
 #pragma unroll
-          for (int t = 0; t < MT; ++t) s[r][t] = 0.f;
+          for (int t = 0; t < MT; ++t)
+            xv[t] = *reinterpret_cast<const float4*>(xb + 4 * ((t * (Sh::KC / 4) + g0 + 2 * w + h) ^ q));
 #pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) {           // 8 weights (one 32-bit word) per row at a time
-          float x[MT][8];
+          for (int i = 0; i < R; ++i) {
+            const float2 v01 = make_float2(lut_at(lut, __byte_perm(eb[i], 0, 0x4440 + 2 * h)),
+                                           lut_at(lut, __byte_perm(ob[i], 0, 0x4440 + 2 * h)));
+            const float2 v23 = make_float2(lut_at(lut, __byte_perm(eb[i], 0, 0x4441 + 2 * h)),
+                                           lut_at(lut, __byte_perm(ob[i], 0, 0x4441 + 2 * h)));
 #pragma unroll
-          for (int t = 0; t < MT; ++t) {
-            const float4 lo = *reinterpret_cast<const float4*>(xs + t * kc + kk + 8 * w4);
-            const float4 hi = *reinterpret_cast<const float4*>(xs + t * kc + kk + 8 * w4 + 4);
-            x[t][0] = lo.x; x[t][1] = lo.y; x[t][2] = lo.z; x[t][3] = lo.w;
-            x[t][4] = hi.x; x[t][5] = hi.y; x[t][6] = hi.z; x[t][7] = hi.w;
-          }
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            const uint32_t wd = w4 == 0 ? q[r].x : (w4 == 1 ? q[r].y : (w4 == 2 ? q[r].z : q[r].w));
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float v = lut[(wd >> (4 * e)) & 15u];
-#pragma unroll
-              for (int t = 0; t < MT; ++t) s[r][t] = fmaf(x[t][e], v, s[r][t]);
+            for (int t = 0; t < MT; ++t) {
+              s[i][t] = __ffma2_rn(make_float2(xv[t].x, xv[t].y), v01, s[i][t]);
+              s[i][t] = __ffma2_rn(make_float2(xv[t].z, xv[t].w), v23, s[i][t]);
             }
           }
         }
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-          for (int t = 0; t < MT; ++t) acc[r][t] = fmaf(a[r], s[r][t], acc[r][t]);
       }
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int t = 0; t < MT; ++t) acc[i][t] = fmaf(ac[i], s[i][t].x + s[i][t].y, acc[i][t]);
     }
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        float v = acc[r][t];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0 && t < M && n0 + r < N) out[static_cast<size_t>(t) * N + n0 + r] = __float2half_rn(v);
-      }
+    if (c + 1 < nchunks) store_chunk(xs[(c + 1) & 1]);
+    __syncthreads();
   }
+
+  // octet sum: lane q == 0 holds the CTA's partial sum of its rows
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      float v = acc[i][t];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      acc[i][t] = v;
+    }
+  if (S == 1) {
+    if (q == 0)
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int t = 0; t < MT; ++t)
+          if (t < M && rows[i] < N) out[static_cast<size_t>(t) * N + rows[i]] = __float2half_rn(acc[i][t]);
+    return;
+  }
+  // S > 1: partial sums to shared memory (the X buffers are free after the last
+  // barrier), then CTA `split` adds the S partials of rows [split, split + 1) * ROWS / S
+  // in rank order, reading the other CTAs' shared memory.
+  float* red = xs[0];
+  if (q == 0)
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+      for (int t = 0; t < MT; ++t) red[((warp * R + i) * 4 + oct) * MT + t] = acc[i][t];
+  cluster_sync();
+  const int r0 = split * Sh::ROWS / S, r1 = (split + 1) * Sh::ROWS / S;
+  const uint32_t red_addr = smem_addr(red);
+  for (int e = tid; e < (r1 - r0) * MT; e += NF_THREADS) {
+    const int rl = r0 + e / MT, t = e % MT;
+    float v = 0.f;
+    for (int r = 0; r < S; ++r) v += ld_shared_cluster_f32(map_to_rank(red_addr + 4u * (rl * MT + t), r));
+    const int n = rb * Sh::ROWS + rl;
+    if (t < M && n < N) out[static_cast<size_t>(t) * N + n] = __float2half_rn(v);
+  }
+  cluster_sync();                                  // keep this CTA's partials alive until all are read
 }
 
 cudaError_t launch_nf4_quantize(const __half* W, int N, int K, uint8_t* packed, float* absmax, int num_sms,
@@ -214,18 +339,78 @@ cudaError_t launch_nf4_dequant(const uint8_t* packed, const float* absmax, int N
   return cudaGetLastError();
 }
 
+namespace {
+
+// Work split of the product: rows per CTA (32R, two choices of R per token
+// count) and the number S of CTAs of a cluster that split K.  An SM's time is
+// taken as proportional to its share of the work, ceil(CTAs / SMs) times the
+// work of one CTA plus one step for its start; the choice closest to an even
+// spread wins (fewer, larger pieces on ties), keeping at least two steps of 256
+// weights per CTA.
+struct Nf4Plan {
+  int R, S, grid;
+};
+
+Nf4Plan nf4_plan(int MT, int N, int K, int num_sms) {
+  const int r_hi = MT <= 2 ? 4 : 2;
+  const int nsteps = (K + NF_STEP - 1) / NF_STEP;
+  Nf4Plan best{r_hi, 1, (N + 32 * r_hi - 1) / (32 * r_hi)};
+  double best_eff = -1.0;
+  for (int R = r_hi; R >= r_hi / 2; R /= 2) {
+    const int rb = (N + 32 * R - 1) / (32 * R);
+    const double ideal = static_cast<double>(N) * K / num_sms;
+    for (int S = 1; S <= 8; ++S) {
+      if (S > 1 && nsteps / S < 2) break;
+      const long long ctas = static_cast<long long>(rb) * S;
+      const long long per_sm = (ctas + num_sms - 1) / num_sms;
+      // a CTA's start (X staging, first loads) is counted as one more step of its rows
+      const double t = static_cast<double>(per_sm) * 32.0 * R * (static_cast<double>(K) / S + NF_STEP);
+      const double eff = ideal / t * (R == r_hi ? 1.0 : 0.97);  // larger R re-reads X less often
+      if (eff > best_eff * 1.02) {
+        best_eff = eff;
+        best = {R, S, static_cast<int>(ctas)};
+      }
+    }
+  }
+  return best;
+}
+
+template <int MT, int R>
+cudaError_t launch_gemv_t(const Nf4Plan& p, const __half* X, int M, const uint8_t* packed, const float* absmax,
+                          int N, int K, const Nf4Tables& tb, __half* out, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(NF_THREADS);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.S > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_nf4_gemv<MT, R>, X, M, packed, absmax, N, K, tb, p.S, out);
+}
+
+}  // namespace
+
 cudaError_t launch_nf4_gemv(const __half* X, int M, const uint8_t* packed, const float* absmax, int N, int K,
                             __half* out, int num_sms, cudaStream_t st) {
   if (M < 1 || M > kNf4MaxTokens) return cudaErrorInvalidValue;
   const Nf4Tables tb = nf4_tables();
-  const int rows = M <= 2 ? 4 : (M <= 4 ? 2 : 1);  // rows per warp of the instantiation below
-  const int groups = (N + NF_WARPS * rows - 1) / (NF_WARPS * rows);
-  const int grid = std::max(1, std::min(groups, num_sms * 4));
-  if (M <= 1) k_nf4_gemv<1, 4><<<grid, NF_THREADS, 0, st>>>(X, M, packed, absmax, N, K, tb, out);
-  else if (M <= 2) k_nf4_gemv<2, 4><<<grid, NF_THREADS, 0, st>>>(X, M, packed, absmax, N, K, tb, out);
-  else if (M <= 4) k_nf4_gemv<4, 2><<<grid, NF_THREADS, 0, st>>>(X, M, packed, absmax, N, K, tb, out);
-  else k_nf4_gemv<8, 1><<<grid, NF_THREADS, 0, st>>>(X, M, packed, absmax, N, K, tb, out);
-  return cudaGetLastError();
+  const int MT = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
+  const Nf4Plan p = nf4_plan(MT, N, K, num_sms);
+  const bool hi = p.R == (MT <= 2 ? 4 : 2);
+  switch (MT) {
+    case 1: return hi ? launch_gemv_t<1, 4>(p, X, M, packed, absmax, N, K, tb, out, st)
+                      : launch_gemv_t<1, 2>(p, X, M, packed, absmax, N, K, tb, out, st);
+    case 2: return hi ? launch_gemv_t<2, 4>(p, X, M, packed, absmax, N, K, tb, out, st)
+                      : launch_gemv_t<2, 2>(p, X, M, packed, absmax, N, K, tb, out, st);
+    case 4: return hi ? launch_gemv_t<4, 2>(p, X, M, packed, absmax, N, K, tb, out, st)
+                      : launch_gemv_t<4, 1>(p, X, M, packed, absmax, N, K, tb, out, st);
+    default: return hi ? launch_gemv_t<8, 2>(p, X, M, packed, absmax, N, K, tb, out, st)
+                       : launch_gemv_t<8, 1>(p, X, M, packed, absmax, N, K, tb, out, st);
+  }
 }
 
 }  // namespace i8lt

@@ -2,10 +2,12 @@
 
 Bit-exact: the packed codes, the block scales and the fp16 dequantised weight.
 The product: |gpu - oracle| <= (64 + K/512) * 2^-23 * sum_k |x_k * w_k| + one fp16
-ulp of the oracle value, a bound derived from the kernel's fp32 evaluation (32-term
-block sums, one scaled accumulation per block half, a 32-lane reduction: at most
-64 + K/512 roundings of size 2^-24 relative to the running sums, each bounded by the
-sum of magnitudes), then one rounding to fp16 on each side.
+ulp of the oracle value, a bound derived from the kernel's fp32 evaluation: per row,
+token and half block two 16-term fused multiply-add chains and their sum, one scaled
+accumulation per half block (at most K/256 per lane), a 3-level sum over the 8 lanes
+of a row and at most 7 additions of cluster partial sums -- fewer than 64 + K/512
+roundings of size 2^-24 relative to the running sums, each bounded by the sum of
+magnitudes -- then one rounding to fp16 on each side.
 """
 
 import numpy as np
@@ -69,8 +71,22 @@ def test_gemv_against_oracle(i8, M, N, K):
     check_gemv(out, X, rp, ra, f"M={M} N={N} K={K}")
 
 
+# Shapes for which the launcher picks each kind of work split: K split over clusters
+# of 1, 2, 3, 4, 6 and 8 CTAs, 32 / 64 / 128 rows per CTA, every token-slot width,
+# ragged N and K (not multiples of the rows per CTA or of 256 weights).
+@pytest.mark.parametrize("M,N,K", [(3, 96, 576), (1, 96, 1088), (6, 1500, 2112), (2, 96, 2112),
+                                   (3, 3000, 2112), (1, 96, 3136), (6, 96, 4160), (7, 200, 4160),
+                                   (2, 4100, 6208), (1, 130, 64), (8, 33, 320)])
+def test_gemv_work_splits(i8, M, N, K):
+    W = wl.weight(740 + N, N, K)
+    X, _ = wl.activation(wl.BASE_SEED + 741 + M, M, K, 3, (8.0, 30.0))
+    rp, ra = nf4.quantize_nf4(W)
+    out = host(i8.i8_nf4_gemv(dev(X), dev(rp), dev(ra)))
+    check_gemv(out, X, rp, ra, f"M={M} N={N} K={K}")
+
+
 @pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672)])
-@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("M", [1, 4, 8])
 def test_gemv_llama70b_sampled_rows(i8, M, N, K):
     """The Llama-70B FFN shapes the bench streams: the GPU quantises and multiplies the whole
     weight; codes, scales and outputs are compared on 256 sampled weight rows (quantisation
@@ -89,6 +105,13 @@ def test_gemv_llama70b_sampled_rows(i8, M, N, K):
 def test_gemv_repeat_is_deterministic(i8):
     W = wl.weight(730, 512, 2048)
     X, _ = wl.activation(wl.BASE_SEED + 731, 3, 2048, 1, (8.0, 30.0))
+    packed, absmax = i8.i8_nf4_quantize(dev(W))
+    a = i8.i8_nf4_gemv(dev(X), packed, absmax)
+    b = i8.i8_nf4_gemv(dev(X), packed, absmax)
+    assert torch.equal(a, b)
+    # a K split over a cluster adds its partial sums in a fixed order too
+    W = wl.weight(732, 8192, 28672)
+    X, _ = wl.activation(wl.BASE_SEED + 733, 8, 28672, 4, (8.0, 30.0))
     packed, absmax = i8.i8_nf4_quantize(dev(W))
     a = i8.i8_nf4_gemv(dev(X), packed, absmax)
     b = i8.i8_nf4_gemv(dev(X), packed, absmax)
