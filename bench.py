@@ -403,11 +403,15 @@ def measure_backward(i8, torch, dev, st, world, dist, reps: int = 20):
             "points": points}
 
 
+GRAPH_CALLS = 20
+
+
 def measure_other(i8, torch, dev, st, world, dist, reps: int = 50):
     """The other workload families, each forward timed alone with CUDA events over `reps`
     back-to-back calls (3 warm-up calls first):
-      - the single 16x1024 -> 1024 linear, launch-latency bound: eager, and the same call
-        captured once in a CUDA graph and replayed;
+      - the single 16x1024 -> 1024 linear, launch-latency bound: eager (back-to-back calls
+        from Python), one call captured in a CUDA graph and replayed, and GRAPH_CALLS calls
+        captured in one graph (time per forward);
       - the OPT-350m-shaped MLP pair at 512 tokens (fc2 fed the ReLU of the GPU's fc1 output,
         computed before timing);
       - the Llama-13B MLP shape 2048x5120 -> 13824 over outlier fractions {0, 0.1, 1, 5} %
@@ -463,11 +467,22 @@ def measure_other(i8, torch, dev, st, world, dist, reps: int = 50):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         run(L, *a)
-    us_graph = timed(graph.replay)
+    us_graph_1 = timed(graph.replay)
+    del graph
+    # a graph of GRAPH_CALLS forwards: the device time per forward once the host no longer
+    # issues each launch (one replay of a one-forward graph is bound by the host call)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(GRAPH_CALLS):
+            run(L, *a)
+    us_graph = timed(graph.replay, n=max(1, reps // 5)) / GRAPH_CALLS
     del graph
     res["single_linear"] = {"shape": f"{L.M}x{L.K}->{L.N}", "outlier_cols": status(a[5]),
                             "us_eager": round(us_eager, 2), "us_graph": round(us_graph, 2),
-                            "TOPS_eager": round(L.ops / us_eager / 1e6, 2)}
+                            "us_graph_one_per_replay": round(us_graph_1, 2),
+                            "graph_calls": GRAPH_CALLS,
+                            "TOPS_eager": round(L.ops / us_eager / 1e6, 2),
+                            "TOPS_graph": round(L.ops / us_graph / 1e6, 2)}
     # OPT-350m MLP pair
     fc1, fc2 = W["C2"].layers
     a1 = prepared("C2", 0, fc1)

@@ -10,6 +10,7 @@ or cannot be loaded, every call raises.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import threading
 
@@ -124,6 +125,20 @@ def _ptr(t):
 
 def _stream(dev):
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+try:  # the current stream's handle without building a Stream object (a per-call cost)
+    _raw_stream = torch._C._cuda_getCurrentRawStream
+except AttributeError:  # pragma: no cover - older torch
+    def _raw_stream(index):
+        return torch.cuda.current_stream(index).cuda_stream
+
+
+def _fits(t, dtype, shape, index):
+    """True when t is a contiguous CUDA tensor of `dtype` and `shape` on device `index`
+    (the cheap test of the per-call path; on False the detailed checks name the problem)."""
+    return (isinstance(t, torch.Tensor) and t.dtype is dtype and t.is_cuda and t.get_device() == index
+            and t.shape == shape and t.is_contiguous())
 
 
 def _need(t, dtype, name, ndim=None):
@@ -362,6 +377,7 @@ def i8_linear8bit_backward_input(dY, Wt, dX=None, status=None):
     return dX
 
 
+@functools.lru_cache(maxsize=1024)
 def i8_linear8bit_workspace_size(M: int, N: int, K: int, max_outlier_cols: int) -> int:
     n = lib().i8_linear8bit_workspace_size(M, N, K, max_outlier_cols)
     if n == 0:
@@ -375,17 +391,32 @@ def i8_linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, out=Non
     _need(X, torch.float16, "X", 2)
     M, K = X.shape
     dev = X.device
-    _need(CB, torch.int8, "CB", 2)
-    N = CB.shape[0]
-    _arg(CB, torch.int8, "CB", (N, K), dev)
-    _arg(SCB, torch.float32, "SCB", (N,), dev)
-    if bias is not None:
-        _arg(bias, torch.float16, "bias", (N,), dev)
-    workspace = _workspace(workspace, dev, i8_linear8bit_workspace_size(M, N, K, max_outlier_cols))
-    out = _out(out, torch.float16, "out", (M, N), dev)
+    index = X.get_device()
+    N = CB.shape[0] if isinstance(CB, torch.Tensor) and CB.dim() == 2 else -1
+    need = i8_linear8bit_workspace_size(M, N, K, max_outlier_cols) if N > 0 else 0
+    if not (_fits(CB, torch.int8, (N, K), index) and _fits(SCB, torch.float32, (N,), index)
+            and (bias is None or _fits(bias, torch.float16, (N,), index))
+            and (out is None or _fits(out, torch.float16, (M, N), index))
+            and (workspace is None or (_fits(workspace, torch.uint8, workspace.shape, index)
+                                       and workspace.dim() == 1))):
+        # the detailed checks raise with a message naming the argument
+        _need(CB, torch.int8, "CB", 2)
+        _arg(CB, torch.int8, "CB", (N, K), dev)
+        _arg(SCB, torch.float32, "SCB", (N,), dev)
+        if bias is not None:
+            _arg(bias, torch.float16, "bias", (N,), dev)
+        if out is not None:
+            _out(out, torch.float16, "out", (M, N), dev)
+        if workspace is not None:
+            _workspace(workspace, dev, need)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
     _check("i8_linear8bit_forward", lib().i8_linear8bit_forward(
-        _ptr(X), _ptr(CB), _ptr(SCB), _ptr(bias), M, N, K, float(threshold), _ptr(out),
-        _ptr(workspace), workspace.numel(), max_outlier_cols, _stream(dev)))
+        X.data_ptr(), CB.data_ptr(), SCB.data_ptr(), None if bias is None else bias.data_ptr(), M, N, K,
+        float(threshold), out.data_ptr(), workspace.data_ptr(), workspace.numel(), max_outlier_cols,
+        _raw_stream(index)))
     return out, workspace
 
 

@@ -111,6 +111,19 @@ struct Units {
   }
 };
 
+// Tile order: bands of kRasterRows tile rows (256 rows of A each); inside a
+// band the rows of one tile column come first, then the next column.  The
+// pairs of one wave then share a few tile rows of A and a few tile columns
+// of B, which the L2 serves to all of them, instead of every row of A.
+constexpr int kRasterRows = 8;
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& tm, int& tn) {
+  const int band = tile / (kRasterRows * num_n);
+  const int r = tile - band * kRasterRows * num_n;
+  const int rows = min(kRasterRows, num_m - band * kRasterRows);  // the last band may be shorter
+  tn = r / rows;
+  tm = band * kRasterRows + (r - tn * rows);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -246,10 +259,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int u = pair; ok && u < U.units && !*s_abort; u += npairs) {
         int tile, half;
         U.at(u, tile, half);
-        const int m0 = (tile % num_m) * (2 * BM) + static_cast<int>(rank) * BM;
+        int tmi, tni;
+        tile_coords(tile, num_m, num_n, tmi, tni);
+        const int m0 = tmi * (2 * BM) + static_cast<int>(rank) * BM;
         // a half tile's 128 columns come as 64 B rows per CTA (the box still
         // carries 128 rows; the MMA reads the first 64)
-        const int nb0 = (tile / num_m) * BN +
+        const int nb0 = tni * BN +
                         (half < 0 ? static_cast<int>(rank) * BNH : half * BNH + static_cast<int>(rank) * (BNH / 2));
         for (int kb = 0; ok && kb < kb_main; ++kb) {
           if (defer && have_prev && kb == j_ins) ok = load_outliers(prev_m0, prev_nb0);
@@ -364,11 +379,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int u = pair; u < U.units; u += npairs, ++it) {  // abort is seen by the wait below
       int tile, half;
       U.at(u, tile, half);
-      const int row_base = (tile % num_m) * (2 * BM) + static_cast<int>(rank) * BM + quad * 32;
+      int tmi, tni;
+      tile_coords(tile, num_m, num_n, tmi, tni);
+      const int row_base = tmi * (2 * BM) + static_cast<int>(rank) * BM + quad * 32;
       // whole tile: 128 columns (4 chunks) per warp; half tile: 64 (2 chunks)
       const int nch = half < 0 ? CHUNKS : CHUNKS / 2;
       const int col_off = col_half * nch * 32;  // TMEM column of this warp's first chunk
-      const int n0 = (tile / num_m) * BN + (half < 0 ? 0 : half * BNH) + col_off;
+      const int n0 = tni * BN + (half < 0 ? 0 : half * BNH) + col_off;
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       // The chunk loop below is deliberately not unrolled: the epilogue runs
@@ -467,7 +484,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
 #pragma unroll 1
       for (int cc = 0; cc < nch; ++cc) {
-        const float sb_c = sb_n, bi_c = bi_n;
+        [[maybe_unused]] const float sb_c = sb_n, bi_c = bi_n;  // unused by the raw and fp16 modes
         uint32_t bf_c[4][2];
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
@@ -513,8 +530,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint32_t halves[2][4][2];
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
-          const int j = cb * 8 + 2 * tq;
-          float sb0 = 0.f, sb1 = 0.f, b0 = 0.f, b1 = 0.f;
+          [[maybe_unused]] const int j = cb * 8 + 2 * tq;
+          [[maybe_unused]] float sb0 = 0.f, sb1 = 0.f, b0 = 0.f, b1 = 0.f;  // stay 0 in the fp16 mode
           if constexpr (!F16) {
             sb0 = __shfl_sync(0xffffffffu, sb_c, j);
             sb1 = __shfl_sync(0xffffffffu, sb_c, j + 1);

@@ -385,9 +385,11 @@ i8_status enqueue_small(const i8_half* X, const int8_t* CB, const float* SCB, co
                         int K, float threshold, i8_half* out, void* workspace, int cap, cudaStream_t st) {
   CUtensorMap tmW;
   if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, CB, K, N, K, 128, 128)) return I8_ERR_CUDA;
+  const int sms = num_sms();
+  if (sms <= 0) return I8_ERR_CUDA;
   return cuda_status(i8lt::launch_linear_small(tmW, reinterpret_cast<const __half*>(X), M, N, K, threshold, cap, SCB,
                                                reinterpret_cast<const __half*>(bias), reinterpret_cast<__half*>(out),
-                                               static_cast<uint32_t*>(workspace), kWaitLimitNs, true, st));
+                                               static_cast<uint32_t*>(workspace), kWaitLimitNs, true, sms, st));
 }
 
 // The forward of one weight on a workspace laid out by ws_layout.
@@ -792,7 +794,8 @@ i8_status i8_linear8bit_forward_multi(const i8_half* X, int M, int K, int G, con
       if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, CB[g], K, N[g], K, 128, 128)) return I8_ERR_CUDA;
       s = cuda_status(i8lt::launch_linear_small(tmW, reinterpret_cast<const __half*>(X), M, N[g], K, threshold, cap,
                                                 SCB[g], reinterpret_cast<const __half*>(bias ? bias[g] : nullptr),
-                                                reinterpret_cast<__half*>(out[g]), w.hdr, kWaitLimitNs, reset, st));
+                                                reinterpret_cast<__half*>(out[g]), w.hdr, kWaitLimitNs, reset, sms,
+                                                st));
       if (s != I8_OK) return s;
       continue;
     }

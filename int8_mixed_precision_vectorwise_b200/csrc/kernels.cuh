@@ -132,10 +132,13 @@ cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap
 // set when reset_status, else only raised to an error).  bias may be null.
 constexpr int kSmallMaxK = 4096;
 constexpr int kSmallListCap = 512;
-size_t linear_small_smem(int K);
+// The grid is ceil(N / 128) clusters of linear_small_split(N, K, num_sms) CTAs,
+// each CTA one slice of K.
+int linear_small_split(int N, int K, int num_sms);
+size_t linear_small_smem(int K, int ks);
 cudaError_t launch_linear_small(const CUtensorMap& tmW, const __half* X, int M, int N, int K, float tau, int cap,
                                 const float* SCB, const __half* bias, __half* out, uint32_t* hdr, uint64_t limit_ns,
-                                bool reset_status, cudaStream_t st);
+                                bool reset_status, int num_sms, cudaStream_t st);
 
 // 4-bit NF4 weight-only product, blocksize 64.  Nf4Tables holds the 16 levels
 // (ascending, level[7] = 0) and the 15 midpoints between neighbours (fp32),

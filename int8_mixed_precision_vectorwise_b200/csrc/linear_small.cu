@@ -6,26 +6,35 @@
 // "LLM.int8() Refactoring: Part 1" (sections "Improved kernels for
 // inference" and "Deprecations").
 //
-// For such sizes the forward's cost is launches and pipeline start-up, not
-// bytes, so everything happens in one grid with no workspace round trip: CTA
-// b owns weight rows [128b, 128b + 128).  It
-//   1. requests its weight tile through a ring of TMA stages (first of all:
-//      the weights do not depend on X);
-//   2. quantises all of X itself (X is at most 16 x 4096 fp16): row absmax
-//      over the elements below the threshold, the outlier-column flags (every
-//      CTA sees every row, so it decides each column alone), codes with the
-//      outlier columns zeroed, written straight into shared memory in the
-//      128B-swizzled K-major layout the tensor core reads, and the sorted
-//      outlier list;
-//   3. runs tcgen05 kind::i8 MMAs (M = 128 weight rows, N = 16 token columns,
-//      int32 accumulator in TMEM) as weight stages land;
-//   4. adds the outlier term X[t, j] * CB[n, j] for the outlier columns from
-//      the staged weight tiles (CUDA cores, fp32, columns in ascending order)
-//      and applies dequant and bias:
+// For such sizes the forward's cost is launches and latency, not bytes, so
+// everything happens in one grid with no workspace round trip, spread over as
+// many SMs as the problem allows: a cluster of KS CTAs (1, 2, 4 or 8) owns
+// weight rows [128t, 128t + 128), and CTA `rank` of it owns a slice of K (whole
+// 128-column boxes).  Each CTA
+//   1. requests its slice of the weight tile through TMA (first of all: the
+//      weights do not depend on X);
+//   2. reads its slice of X: per row the absmax over the elements below the
+//      threshold, and the outlier-column flags of its columns; the sorted list
+//      of its outlier columns;
+//   3. exchanges the row maxima and outlier counts with the other CTAs of the
+//      cluster through distributed shared memory: the row scale is the max
+//      over all slices, and a column's position in the forward's ascending
+//      outlier list is its CTA's offset plus its index in the CTA's list;
+//   4. writes its codes (outlier columns zeroed) straight into shared memory in
+//      the 128B-swizzled K-major layout the tensor core reads, and runs tcgen05
+//      kind::i8 MMAs (M = 128 weight rows, N = 16 token columns, int32
+//      accumulator in TMEM) as the weight boxes land;
+//   5. computes the outlier term X[t, j] * CB[n, j] of its outlier columns from
+//      the staged weight boxes (CUDA cores, fp32, ascending columns);
+//   6. publishes its int32 partial accumulator and fp32 outlier partial sums;
+//      after a cluster barrier CTA `rank` adds, for rows
+//      [rank * 128 / KS, (rank + 1) * 128 / KS), the KS partials in rank order
+//      (the int32 sum is exact) and applies dequant and bias:
 //        out[t, n] = fp16(C * SCA[t] * SCB[n] / 127^2 + bias[n] + (SCB[n] / 127) * D).
-// Block 0 writes the status word and the outlier counts.  Every wait is
-// bounded by a time limit; on expiry the status becomes I8_ERR_TIMEOUT and
-// the CTA leaves after its in-flight copies and MMAs have completed.
+// Block 0 writes the status word and the outlier counts.  Every mbarrier wait
+// is bounded by a time limit; on expiry the status becomes I8_ERR_TIMEOUT and
+// the CTA still takes both cluster barriers (after its in-flight copies and
+// MMAs have completed), so its peers never wait for it for good.
 #include <cuda_fp16.h>
 
 #include <atomic>
@@ -37,27 +46,30 @@ namespace i8lt {
 
 namespace {
 
-constexpr int LM = 128;                       // weight rows per CTA (MMA M)
+constexpr int LM = 128;                       // weight rows per cluster (MMA M)
 constexpr int LT = kDecodeMaxTokens;          // token columns (MMA N), zero padded
 constexpr int LBOX = LM * 128;                // one 128-byte-deep weight box: 16 KB
 constexpr int LSB = 2;                        // weight boxes per ring stage
 constexpr int LSTAGE = LSB * LBOX;            // 32 KB
-constexpr int LRS = 4;                        // ring stages
+constexpr int LRS = 4;                        // ring stages at most
 constexpr int LCA_BOX = LT * 128;             // one 128-byte-deep box of the 16 code rows: 2 KB
 constexpr int LTHREADS = 256;
 constexpr int LPU = 8;                        // X vectors per thread in flight while quantising
+constexpr int LMAXKS = 8;                     // CTAs per cluster at most
 constexpr uint32_t LTMEM_COLS = 32;
 constexpr unsigned kAllLanes = 0xffffffffu;
 
+// Shared memory of a CTA whose slice has nbl boxes.
 struct SmallLayout {
-  int ca_off, sbm_off, list_off, misc_off, bar_off, total;
-  __host__ __device__ SmallLayout(int K) {
-    const int nbox = (K + 127) / 128;
-    ca_off = LRS * LSTAGE;
-    sbm_off = ca_off + nbox * LCA_BOX;
-    list_off = sbm_off + ((K + 31) / 32) * 4;
-    misc_off = list_off + kSmallListCap * 4;
-    bar_off = (misc_off + 3 * LT * 4 + 16 + 7) & ~7;
+  int stages, ca_off, sbm_off, list_off, red_off, misc_off, bar_off, total;
+  __host__ __device__ explicit SmallLayout(int nbl) {
+    stages = (nbl + LSB - 1) / LSB < LRS ? (nbl + LSB - 1) / LSB : LRS;
+    ca_off = stages * LSTAGE;
+    sbm_off = ca_off + nbl * LCA_BOX;
+    list_off = sbm_off + nbl * 16;                            // 4 bitmap words per box
+    red_off = list_off + kSmallListCap * 4;                   // int32 C [128][16] and fp32 D [128][16]
+    misc_off = red_off + 2 * LM * LT * 4;
+    bar_off = (misc_off + 4 * LT * 4 + 32 + 7) & ~7;
     total = bar_off + (2 * LRS + 1) * 8 + 1024;  // + slack to align the ring to 1024 bytes
   }
 };
@@ -68,36 +80,61 @@ __device__ __forceinline__ uint32_t small_code(float x, float r) {
   return q;
 }
 
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 }  // namespace
 
-size_t linear_small_smem(int K) { return static_cast<size_t>(SmallLayout(K).total); }
+size_t linear_small_smem(int K, int ks) {
+  const int nbox = (K + 127) / 128;
+  return static_cast<size_t>(SmallLayout((nbox + ks - 1) / ks).total);
+}
+
+int linear_small_split(int N, int K, int num_sms) {
+  const int ntile = (N + LM - 1) / LM, nbox = (K + 127) / 128;
+  int ks = LMAXKS;
+  while (ks > 1 && (ks > nbox || static_cast<long long>(ntile) * ks > num_sms)) ks /= 2;
+  return ks;
+}
 
 __global__ void __launch_bounds__(LTHREADS, 1)
     k_linear_small(const __grid_constant__ CUtensorMap tmW, const __half* __restrict__ X, int M, int N, int K,
                    float tau, int cap, const float* __restrict__ SCB, const __half* __restrict__ bias,
-                   __half* __restrict__ out, uint32_t* hdr, uint64_t limit_ns, int reset_status) {
+                   __half* __restrict__ out, uint32_t* hdr, uint64_t limit_ns, int reset_status, int KS) {
   extern __shared__ uint8_t lsm_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
-  const SmallLayout Lay(K);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = KS > 1 ? static_cast<int>(blockIdx.x % KS) : 0;
+  const int n0 = (KS > 1 ? static_cast<int>(blockIdx.x / KS) : static_cast<int>(blockIdx.x)) * LM;
+  const int nbox = (K + 127) / 128;
+  const int kb0 = rank * nbox / KS, kb1 = (rank + 1) * nbox / KS;  // this CTA's boxes
+  const int nbl = kb1 - kb0;
+  const int nbl_max = (nbox + KS - 1) / KS;                         // the layout is the same in every CTA
+  const SmallLayout Lay(nbl_max);
   uint8_t* ring = smem;
   uint8_t* ca = smem + Lay.ca_off;
   uint32_t* sbm = reinterpret_cast<uint32_t*>(smem + Lay.sbm_off);
   int32_t* s_list = reinterpret_cast<int32_t*>(smem + Lay.list_off);
-  uint32_t* s_rowmax = reinterpret_cast<uint32_t*>(smem + Lay.misc_off);  // fp32 bits of maxima
+  int32_t* red_c = reinterpret_cast<int32_t*>(smem + Lay.red_off);
+  float* red_d = reinterpret_cast<float*>(red_c + LM * LT);
+  uint32_t* s_rowmax = reinterpret_cast<uint32_t*>(smem + Lay.misc_off);  // this slice's maxima (fp32 bits)
   float* s_r = reinterpret_cast<float*>(s_rowmax + LT);
   float* s_sa = s_r + LT;
-  int* s_cnt = reinterpret_cast<int*>(s_sa + LT);        // [0] outlier columns found
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_cnt + 1);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(s_cnt + 2);
+  int* s_cnt = reinterpret_cast<int*>(s_sa + LT);         // [0] this slice's outlier columns
+  int* s_base = s_cnt + 1;                                // [0] columns in earlier slices, [1] in all
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_cnt + 3);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_cnt + 4);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay.bar_off);
   uint64_t* empty = full + LRS;
   uint64_t* acc_full = empty + LRS;
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * LM;
-  const int nbox = (K + 127) / 128;                 // 128-byte k-boxes
-  const int nstage = (nbox + LSB - 1) / LSB;
-  const int nvec = K >> 3, nwords = (K + 31) >> 5;
+  const int k0 = kb0 * 128, k1 = min(K, kb1 * 128);       // this CTA's columns
+  const int nstage = (nbl + LSB - 1) / LSB;
+  const int RS = Lay.stages;
+  const int nvec = (k1 - k0) >> 3, nwords = nbl * 4;
   const bool use_tau = tau > 0.f;
 
   if (tid == 0) {
@@ -117,40 +154,41 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   if (tid < LT) s_rowmax[tid] = 0u;
   {  // zero the code tile: rows past M and bytes past K must be 0 for the MMA
     uint4* z = reinterpret_cast<uint4*>(ca);
-    for (int i = tid; i < nbox * LCA_BOX / 16; i += LTHREADS) z[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < nbl * LCA_BOX / 16; i += LTHREADS) z[i] = make_uint4(0, 0, 0, 0);
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
 
-  // the weight tile does not depend on X: request the first stages now
+  // the weight slice does not depend on X: request the first stages now
   uint32_t filled = 0, fill_parity = 0;
   if (tid == 0) {
     tma_prefetch_desc(&tmW);
-    for (int st = 0; st < nstage && st < LRS; ++st) {
-      const int b0 = st * LSB, nb = min(LSB, nbox - b0);
+    for (int st = 0; st < nstage && st < RS; ++st) {
+      const int b0 = st * LSB, nb = min(LSB, nbl - b0);
       mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nb * LBOX));
       filled |= 1u << st;
-      for (int b = 0; b < nb; ++b) tma_load_2d(ring + st * LSTAGE + b * LBOX, &tmW, &full[st], (b0 + b) * 128, n0);
+      for (int b = 0; b < nb; ++b)
+        tma_load_2d(ring + st * LSTAGE + b * LBOX, &tmW, &full[st], (kb0 + b0 + b) * 128, n0);
     }
   }
 
-  // ---------------------------------------------------------------- quantise X (all threads)
+  // ---------------------------------------------------------------- this slice of X (all threads)
   // Items (row, 8-column vector) in chunks of LPU per thread: all LPU loads of
-  // a chunk are issued before any is used.  When X fits in one chunk it stays
-  // in registers for pass 2; otherwise pass 2 reads each chunk again (from L1/L2).
+  // a chunk are issued before any is used.  When the slice fits in one chunk it
+  // stays in registers for the codes; otherwise they read each chunk again.
   const int items = M * nvec;
   const bool one_chunk = items <= LPU * LTHREADS;
   uint4 xv[LPU];
-  for (int base = 0; base < items; base += LPU * LTHREADS) {   // pass 1: row maxima below the threshold, column flags
+  for (int base = 0; base < items; base += LPU * LTHREADS) {   // row maxima below the threshold, column flags
 #pragma unroll
     for (int u = 0; u < LPU; ++u) {
       const int it = base + u * LTHREADS + tid;
       xv[u] = make_uint4(0, 0, 0, 0);
       if (it < items) {
         const int r = it / nvec;
-        xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + (it - r * nvec));
+        xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + k0) + (it - r * nvec));
       }
     }
 #pragma unroll
@@ -186,20 +224,63 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     }
   }
   __syncthreads();
+  if (warp == 0) {   // this slice's sorted outlier list (ascending columns)
+    const int per = (nwords + 31) / 32;
+    const int w0 = min(lane * per, nwords), w1 = min(w0 + per, nwords);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(sbm[w]);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kAllLanes, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = incl - cnt;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = sbm[w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (pos < kSmallListCap) s_list[pos] = k0 + 32 * w + b;
+        ++pos;
+      }
+    }
+    if (lane == 31) *s_cnt = incl;
+  }
+  // ---------------------------------------------------------------- exchange with the cluster
+  if (KS > 1) cluster_sync(); else __syncthreads();
   if (tid < LT) {
-    const float amax = tid < M ? __uint_as_float(s_rowmax[tid]) : 0.f;
+    uint32_t m = s_rowmax[tid];
+    if (KS > 1) {
+      const uint32_t a = smem_addr(s_rowmax + tid);
+      for (int r = 0; r < KS; ++r) m = max(m, ld_cluster_u32(map_to_rank(a, r)));
+    }
+    const float amax = tid < M ? __uint_as_float(m) : 0.f;
     s_r[tid] = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
     s_sa[tid] = amax * (1.0f / 16129.0f);
+  } else if (tid == LT) {
+    int before = 0, all = *s_cnt;
+    if (KS > 1) {
+      const uint32_t a = smem_addr(s_cnt);
+      all = 0;
+      for (int r = 0; r < KS; ++r) {
+        const int c = static_cast<int>(ld_cluster_u32(map_to_rank(a, r)));
+        if (r < rank) before += c;
+        all += c;
+      }
+    }
+    s_base[0] = before;
+    s_base[1] = all;
   }
   __syncthreads();
-  for (int base = 0; base < items; base += LPU * LTHREADS) {   // pass 2: codes into the swizzled K-major tile
+  for (int base = 0; base < items; base += LPU * LTHREADS) {   // codes into the swizzled K-major tile
     if (!one_chunk) {
 #pragma unroll
       for (int u = 0; u < LPU; ++u) {
         const int it = base + u * LTHREADS + tid;
         if (it < items) {
           const int r = it / nvec;
-          xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + (it - r * nvec));
+          xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + k0) + (it - r * nvec));
         }
       }
     }
@@ -225,38 +306,17 @@ __global__ void __launch_bounds__(LTHREADS, 1)
         for (int e = 0; e < 8; ++e)
           if (fl & (1u << e)) w[e >> 2] &= ~(0xffu << ((e & 3) * 8));
       }
-      // byte kk = 8v of row r: box kk / 128, 16-byte chunk q = (kk % 128) / 16 stored at q ^ (r % 8)
+      // byte kk = 8v of row r in the slice: box kk / 128, 16-byte chunk q = (kk % 128) / 16 stored at q ^ (r % 8)
       const int kk = 8 * v, box = kk >> 7, q = (kk & 127) >> 4;
       *reinterpret_cast<uint2*>(ca + box * LCA_BOX + r * 128 + ((q ^ (r & 7)) << 4) + (kk & 15)) = make_uint2(w[0], w[1]);
     }
   }
-  if (warp == 0) {   // the sorted outlier list (ascending columns)
-    const int per = (nwords + 31) / 32;
-    const int w0 = min(lane * per, nwords), w1 = min(w0 + per, nwords);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(sbm[w]);
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kAllLanes, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pos = incl - cnt;
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = sbm[w];
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (pos < kSmallListCap) s_list[pos] = 32 * w + b;
-        ++pos;
-      }
-    }
-    if (lane == 31) *s_cnt = incl;
-  }
   fence_async_shared();   // the code tile was written by threads; the tensor core reads it
   __syncthreads();
-  const int total = use_tau ? *s_cnt : 0;
+  const int total = use_tau ? s_base[1] : 0;
   const int used = min(total, min(cap, kSmallListCap));
+  // entries [0, lused) of this slice's list are in the forward's first `used` columns
+  const int lused = use_tau ? max(0, min(*s_cnt, used - s_base[0])) : 0;
   if (blockIdx.x == 0 && tid == 0) {
     if (reset_status)
       hdr[0] = total > cap ? kStatusOutlierOverflow : kStatusOk;
@@ -266,22 +326,24 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     hdr[2] = static_cast<uint32_t>(total);
   }
 
+  const int quad = warp & 3, row = quad * 32 + lane;    // epilogue warps 4..7: weight row of the tile
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer (the rest of the tile)
+    // ---------------------------------------------------------------- TMA producer (the rest of the slice)
     if (lane == 0) {
-      for (int st = LRS; st < nstage; ++st) {
-        const int s = st % LRS;
-        const uint32_t use = static_cast<uint32_t>(st / LRS);
+      for (int st = RS; st < nstage; ++st) {
+        const int s = st % RS;
+        const uint32_t use = static_cast<uint32_t>(st / RS);
         if (!mbar_wait_bounded(&empty[s], (use - 1) & 1u, s_abort, hdr, limit_ns)) break;
-        const int b0 = st * LSB, nb = min(LSB, nbox - b0);
+        const int b0 = st * LSB, nb = min(LSB, nbl - b0);
         mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nb * LBOX));
         filled |= 1u << s;
         fill_parity = (fill_parity & ~(1u << s)) | ((use & 1u) << s);
-        for (int b = 0; b < nb; ++b) tma_load_2d(ring + s * LSTAGE + b * LBOX, &tmW, &full[s], (b0 + b) * 128, n0);
+        for (int b = 0; b < nb; ++b)
+          tma_load_2d(ring + s * LSTAGE + b * LBOX, &tmW, &full[s], (kb0 + b0 + b) * 128, n0);
       }
       if (*s_abort) {
         int never = 0;
-        for (int s = 0; s < LRS; ++s)
+        for (int s = 0; s < RS; ++s)
           if (filled & (1u << s)) mbar_wait_bounded(&full[s], (fill_parity >> s) & 1u, &never, nullptr, limit_ns);
       }
     }
@@ -291,10 +353,10 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_i8_s32(LM, LT);
       for (int st = 0; st < nstage && !*s_abort; ++st) {
-        const int s = st % LRS;
-        if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(st / LRS) & 1u, s_abort, hdr, limit_ns)) break;
+        const int s = st % RS;
+        if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>(st / RS) & 1u, s_abort, hdr, limit_ns)) break;
         tc_fence_after_sync();
-        const int b0 = st * LSB, nb = min(LSB, nbox - b0);
+        const int b0 = st * LSB, nb = min(LSB, nbl - b0);
         for (int b = 0; b < nb; ++b) {
           const uint64_t adesc = smem_desc_k_sw128(smem_addr(ring + s * LSTAGE + b * LBOX));
           const uint64_t bdesc = smem_desc_k_sw128(smem_addr(ca + (b0 + b) * LCA_BOX));
@@ -308,30 +370,30 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------------------------------------------------------- outlier term + epilogue
-    // thread = weight row r of the tile (TMEM lane r: warps 4..7 read lane quadrants 0..3)
-    const int quad = warp & 3, r = quad * 32 + lane, n = n0 + r;
+    // ---------------------------------------------------------------- outlier term + partial results
+    // thread = weight row `row` of the tile (TMEM lane row: warps 4..7 read lane quadrants 0..3)
     float d[LT];
 #pragma unroll
     for (int t = 0; t < LT; ++t) d[t] = 0.f;
     int cur = 0;
     bool ok = true;
     for (int st = 0; st < nstage; ++st) {
-      const int s = st % LRS;
+      const int s = st % RS;
       int got = 0;
-      if (lane == 0) got = mbar_wait_bounded(&full[s], static_cast<uint32_t>(st / LRS) & 1u, s_abort, hdr, limit_ns);
+      if (lane == 0) got = mbar_wait_bounded(&full[s], static_cast<uint32_t>(st / RS) & 1u, s_abort, hdr, limit_ns);
       if (!__shfl_sync(kAllLanes, got, 0)) {
         ok = false;
         break;
       }
       const uint8_t* sa = ring + s * LSTAGE;
-      const int kbeg = st * LSB * 128;
-      while (cur < used) {
+      const int kbeg = k0 + st * LSB * 128;
+      while (cur < lused) {
         const int j = s_list[cur];
         const int kk = j - kbeg;
         if (kk >= LSB * 128) break;
         const int box = kk >> 7, b = kk & 127;
-        const float w = static_cast<float>(static_cast<int8_t>(sa[box * LBOX + r * 128 + (((b >> 4) ^ (r & 7)) << 4) + (b & 15)]));
+        const float w =
+            static_cast<float>(static_cast<int8_t>(sa[box * LBOX + row * 128 + (((b >> 4) ^ (row & 7)) << 4) + (b & 15)]));
 #pragma unroll
         for (int t = 0; t < LT; ++t)
           if (t < M) d[t] = fmaf(__half2float(X[static_cast<size_t>(t) * K + j]), w, d[t]);
@@ -342,20 +404,33 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     }
     int acc = 0;
     if (ok && lane == 0) acc = mbar_wait_bounded(acc_full, 0, s_abort, hdr, limit_ns) ? 1 : 0;
+    uint32_t c[LT];
+#pragma unroll
+    for (int t = 0; t < LT; ++t) c[t] = 0u;
     if (__shfl_sync(kAllLanes, acc, 0)) {
       tc_fence_after_sync();
-      uint32_t c[LT];
       tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(quad * 32) << 16), c);
       tmem_wait_ld();
+    }
+    if (KS == 1) {
+      const int n = n0 + row;
       if (n < N) {
         const float sb = __ldg(SCB + n);
         const float bv = bias != nullptr ? __half2float(bias[n]) : 0.f;
 #pragma unroll
         for (int t = 0; t < LT; ++t) {
           if (t >= M) break;
-          const float y = fmaf(d[t], sb * (1.0f / 127.0f), fmaf(static_cast<float>(static_cast<int32_t>(c[t])), s_sa[t] * sb, bv));
+          const float y = fmaf(d[t], sb * (1.0f / 127.0f),
+                               fmaf(static_cast<float>(static_cast<int32_t>(c[t])), s_sa[t] * sb, bv));
           out[static_cast<size_t>(t) * N + n] = __float2half_rn(y);
         }
+      }
+    } else {
+      // partials of row `row`: 16 int32 and 16 fp32
+#pragma unroll
+      for (int ch = 0; ch < LT / 4; ++ch) {
+        *reinterpret_cast<uint4*>(red_c + row * LT + 4 * ch) = make_uint4(c[4 * ch], c[4 * ch + 1], c[4 * ch + 2], c[4 * ch + 3]);
+        *reinterpret_cast<float4*>(red_d + row * LT + 4 * ch) = make_float4(d[4 * ch], d[4 * ch + 1], d[4 * ch + 2], d[4 * ch + 3]);
       }
     }
   }
@@ -365,6 +440,28 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     int never = 0;
     if (lane == 0) mbar_wait_bounded(acc_full, 0, &never, nullptr, limit_ns);
     __syncwarp();
+  }
+  if (KS > 1) {
+    // ---------------------------------------------------------------- sum of the cluster's partials
+    cluster_sync();
+    const int r0 = rank * LM / KS, r1 = (rank + 1) * LM / KS;
+    const uint32_t ac = smem_addr(red_c), ad = smem_addr(red_d);
+    for (int e = tid; e < (r1 - r0) * LT; e += LTHREADS) {
+      const int rl = r0 + e / LT, t = e % LT, n = n0 + rl;
+      if (t >= M || n >= N) continue;
+      int32_t csum = 0;
+      float dsum = 0.f;
+      const uint32_t off = 4u * static_cast<uint32_t>(rl * LT + t);
+      for (int r = 0; r < KS; ++r) {
+        csum += static_cast<int32_t>(ld_cluster_u32(map_to_rank(ac + off, r)));
+        dsum += __uint_as_float(ld_cluster_u32(map_to_rank(ad + off, r)));
+      }
+      const float sb = __ldg(SCB + n);
+      const float bv = bias != nullptr ? __half2float(bias[n]) : 0.f;
+      const float y = fmaf(dsum, sb * (1.0f / 127.0f), fmaf(static_cast<float>(csum), s_sa[t] * sb, bv));
+      out[static_cast<size_t>(t) * N + n] = __float2half_rn(y);
+    }
+    cluster_sync();   // this CTA's partials stay in place until every CTA has read them
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -376,21 +473,33 @@ __global__ void __launch_bounds__(LTHREADS, 1)
 
 cudaError_t launch_linear_small(const CUtensorMap& tmW, const __half* X, int M, int N, int K, float tau, int cap,
                                 const float* SCB, const __half* bias, __half* out, uint32_t* hdr, uint64_t limit_ns,
-                                bool reset_status, cudaStream_t st) {
-  const size_t smem = linear_small_smem(K);
+                                bool reset_status, int num_sms, cudaStream_t st) {
+  const int ks = linear_small_split(N, K, num_sms);
+  const size_t smem = linear_small_smem(K, ks);
   static std::atomic<bool> attr_done[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(k_linear_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(linear_small_smem(kSmallMaxK)));
+                                         static_cast<int>(linear_small_smem(kSmallMaxK, 1)));
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
   }
-  const int grid = (N + LM - 1) / LM;
-  k_linear_small<<<grid, LTHREADS, smem, st>>>(tmW, X, M, N, K, tau, cap, SCB, bias, out, hdr, limit_ns,
-                                                reset_status ? 1 : 0);
-  return cudaGetLastError();
+  const int ntile = (N + LM - 1) / LM;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ntile * ks);
+  cfg.blockDim = dim3(LTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ks > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_linear_small, tmW, X, M, N, K, tau, cap, SCB, bias, out, hdr, limit_ns,
+                            reset_status ? 1 : 0, ks);
 }
 
 }  // namespace i8lt

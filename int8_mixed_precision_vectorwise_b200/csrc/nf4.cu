@@ -344,9 +344,9 @@ namespace {
 // Work split of the product: rows per CTA (32R, two choices of R per token
 // count) and the number S of CTAs of a cluster that split K.  An SM's time is
 // taken as proportional to its share of the work, ceil(CTAs / SMs) times the
-// work of one CTA plus one step for its start; the choice closest to an even
-// spread wins (fewer, larger pieces on ties), keeping at least two steps of 256
-// weights per CTA.
+// work of one CTA plus one step for its start, times the shared-memory
+// wavefronts per 32 weights (1 + MT / R); the smallest estimate wins (fewer,
+// larger pieces on ties), keeping at least two steps of 256 weights per CTA.
 struct Nf4Plan {
   int R, S, grid;
 };
@@ -363,9 +363,13 @@ Nf4Plan nf4_plan(int MT, int N, int K, int num_sms) {
       if (S > 1 && nsteps / S < 2) break;
       const long long ctas = static_cast<long long>(rb) * S;
       const long long per_sm = (ctas + num_sms - 1) / num_sms;
-      // a CTA's start (X staging, first loads) is counted as one more step of its rows
-      const double t = static_cast<double>(per_sm) * 32.0 * R * (static_cast<double>(K) / S + NF_STEP);
-      const double eff = ideal / t * (R == r_hi ? 1.0 : 0.97);  // larger R re-reads X less often
+      // a CTA's start (X staging, first loads) is counted as one more step of its rows;
+      // per 32 weights the lookups take one shared-memory wavefront and the X values
+      // MT / R more (each lane reads MT values per k and uses them for R rows)
+      // (an SM given a single CTA, 8 warps, hides latency about half as well)
+      const double t = static_cast<double>(per_sm) * 32.0 * R * (static_cast<double>(K) / S + NF_STEP) *
+                       (1.0 + static_cast<double>(MT) / R) * (per_sm < 2 ? 2.0 : 1.0);
+      const double eff = ideal / t * (1.0 + static_cast<double>(MT) / r_hi);
       if (eff > best_eff * 1.02) {
         best_eff = eff;
         best = {R, S, static_cast<int>(ctas)};

@@ -307,13 +307,16 @@ def test_selftest_bounded_wait_times_out(i8):
 
 # ------------------------------------------------------------------ one-launch small forward
 SMALL_SHAPES = [
-    # M, N, K, planted columns, threshold, bias   (all take the one-launch kernel)
+    # M, N, K, planted columns, threshold, bias   (all take the one-launch kernel; on 148 SMs
+    # K is split over clusters of 8, 8, 2, 4, 8, 8, 1 and 8 CTAs)
     (16, 1024, 1024, 2, 6.0, True),     # the single-linear workload
     (1, 1024, 4096, 3, 6.0, False),     # one token, the longest row the kernel takes
     (5, 300, 272, 4, 6.0, True),        # ragged N (a partial weight tile) and ragged K (a partial box)
     (16, 4096, 1024, 0, 6.0, True),     # 32 tiles, no outliers
     (9, 2048, 2064, 40, 6.0, False),    # many outlier columns spread over every stage
     (12, 512, 1024, 3, 0.0, True),      # threshold 0
+    (4, 16384, 512, 2, 6.0, True),      # 128 tiles: one CTA per tile (no K split)
+    (7, 2048, 1152, 9, 6.0, True),      # 9 boxes over a cluster of 8: one CTA takes two
 ]
 
 
