@@ -10,7 +10,6 @@ or cannot be loaded, every call raises.
 from __future__ import annotations
 
 import ctypes
-import functools
 import os
 import threading
 
@@ -132,6 +131,11 @@ try:  # the current stream's handle without building a Stream object (a per-call
 except AttributeError:  # pragma: no cover - older torch
     def _raw_stream(index):
         return torch.cuda.current_stream(index).cuda_stream
+
+
+def _stream_handle(index):
+    """The current stream of CUDA device `index`, as the integer handle the C ABI takes."""
+    return _raw_stream(index)
 
 
 def _fits(t, dtype, shape, index):
@@ -377,12 +381,19 @@ def i8_linear8bit_backward_input(dY, Wt, dX=None, status=None):
     return dX
 
 
-@functools.lru_cache(maxsize=1024)
+_ws_sizes: dict = {}
+
+
 def i8_linear8bit_workspace_size(M: int, N: int, K: int, max_outlier_cols: int) -> int:
-    n = lib().i8_linear8bit_workspace_size(M, N, K, max_outlier_cols)
-    if n == 0:
-        raise I8Error("i8_linear8bit_workspace_size", 1)
-    return int(n)
+    key = (id(lib()), M, N, K, max_outlier_cols)   # remembered per shape (a per-call cost otherwise)
+    n = _ws_sizes.get(key)
+    if n is None:
+        n = int(lib().i8_linear8bit_workspace_size(M, N, K, max_outlier_cols))
+        if n == 0:
+            raise I8Error("i8_linear8bit_workspace_size", 1)
+        if len(_ws_sizes) < 4096:
+            _ws_sizes[key] = n
+    return n
 
 
 def i8_linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, out=None, workspace=None,
@@ -416,7 +427,7 @@ def i8_linear8bit_forward(X, CB, SCB, bias=None, threshold: float = 6.0, out=Non
     _check("i8_linear8bit_forward", lib().i8_linear8bit_forward(
         X.data_ptr(), CB.data_ptr(), SCB.data_ptr(), None if bias is None else bias.data_ptr(), M, N, K,
         float(threshold), out.data_ptr(), workspace.data_ptr(), workspace.numel(), max_outlier_cols,
-        _raw_stream(index)))
+        _stream_handle(index)))
     return out, workspace
 
 

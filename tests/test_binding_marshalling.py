@@ -45,6 +45,7 @@ def fake(monkeypatch):
 
     monkeypatch.setattr(b, "_need", need_on_any_device)
     monkeypatch.setattr(b, "_stream", lambda dev: None)
+    monkeypatch.setattr(b, "_stream_handle", lambda index: None)
     monkeypatch.setattr(b, "lib", lambda: lib)
     return lib
 
