@@ -16,24 +16,29 @@
 //   2. reads its slice of X: per row the absmax over the elements below the
 //      threshold, and the outlier-column flags of its columns; the sorted list
 //      of its outlier columns;
-//   3. exchanges the row maxima and outlier counts with the other CTAs of the
-//      cluster through distributed shared memory: the row scale is the max
-//      over all slices, and a column's position in the forward's ascending
-//      outlier list is its CTA's offset plus its index in the CTA's list;
-//   4. writes its codes (outlier columns zeroed) straight into shared memory in
-//      the 128B-swizzled K-major layout the tensor core reads, and runs tcgen05
-//      kind::i8 MMAs (M = 128 weight rows, N = 16 token columns, int32
-//      accumulator in TMEM) as the weight boxes land;
+//   3. stores its row maxima and outlier count into every CTA of the cluster
+//      (distributed shared memory, no remote loads); after one cluster barrier
+//      each CTA has them locally: the row scale is the max over all slices, and
+//      a column's position in the forward's ascending outlier list is its CTA's
+//      offset plus its index in the CTA's list;
+//   4. writes its codes (outlier columns zeroed; their X values kept in shared
+//      memory for step 5) straight into shared memory in the 128B-swizzled
+//      K-major layout the tensor core reads, and runs tcgen05 kind::i8 MMAs
+//      (M = 128 weight rows, N = 16 token columns, int32 accumulator in TMEM) as
+//      the weight boxes land;
 //   5. computes the outlier term X[t, j] * CB[n, j] of its outlier columns from
 //      the staged weight boxes (CUDA cores, fp32, ascending columns);
-//   6. publishes its int32 partial accumulator and fp32 outlier partial sums;
-//      after a cluster barrier CTA `rank` adds, for rows
-//      [rank * 128 / KS, (rank + 1) * 128 / KS), the KS partials in rank order
-//      (the int32 sum is exact) and applies dequant and bias:
+//   6. stores its int32 partial accumulator and fp32 outlier partial sums of
+//      each row into the CTA that finishes the row (CTA `rank` owns rows
+//      [rank * 128 / KS, (rank + 1) * 128 / KS)); after a second cluster barrier
+//      that CTA adds the KS partials in rank order (the int32 sum is exact) and
+//      applies dequant and bias:
 //        out[t, n] = fp16(C * SCA[t] * SCB[n] / 127^2 + bias[n] + (SCB[n] / 127) * D).
+// A first cluster barrier, split into an arrive at the start and a wait before
+// the first remote store, makes sure every CTA of the cluster has started.
 // Block 0 writes the status word and the outlier counts.  Every mbarrier wait
 // is bounded by a time limit; on expiry the status becomes I8_ERR_TIMEOUT and
-// the CTA still takes both cluster barriers (after its in-flight copies and
+// the CTA still takes every cluster barrier (after its in-flight copies and
 // MMAs have completed), so its peers never wait for it for good.
 #include <cuda_fp16.h>
 
@@ -54,21 +59,27 @@ constexpr int LSTAGE = LSB * LBOX;            // 32 KB
 constexpr int LRS = 4;                        // ring stages at most
 constexpr int LCA_BOX = LT * 128;             // one 128-byte-deep box of the 16 code rows: 2 KB
 constexpr int LTHREADS = 256;
-constexpr int LPU = 8;                        // X vectors per thread in flight while quantising
+constexpr int LPU = 4;                        // X vectors per thread in flight while quantising
 constexpr int LMAXKS = 8;                     // CTAs per cluster at most
 constexpr uint32_t LTMEM_COLS = 32;
 constexpr unsigned kAllLanes = 0xffffffffu;
 
-// Shared memory of a CTA whose slice has nbl boxes.
+// Shared memory of a CTA whose slice has nbl boxes, in a cluster of ks CTAs.  With
+// ks > 1 it also receives the other CTAs' row maxima and outlier counts (xch) and, for
+// its 128 / ks rows, their partial sums (red: int32 C and fp32 D, [ks][128 / ks][16]).
 struct SmallLayout {
-  int stages, ca_off, sbm_off, list_off, red_off, misc_off, bar_off, total;
-  __host__ __device__ explicit SmallLayout(int nbl) {
+  int stages, ca_off, sbm_off, wpre_off, list_off, xo_off, sc_off, xch_off, red_off, misc_off, bar_off, total;
+  __host__ __device__ SmallLayout(int nbl, int ks) {
     stages = (nbl + LSB - 1) / LSB < LRS ? (nbl + LSB - 1) / LSB : LRS;
     ca_off = stages * LSTAGE;
     sbm_off = ca_off + nbl * LCA_BOX;
-    list_off = sbm_off + nbl * 16;                            // 4 bitmap words per box
-    red_off = list_off + kSmallListCap * 4;                   // int32 C [128][16] and fp32 D [128][16]
-    misc_off = red_off + 2 * LM * LT * 4;
+    wpre_off = sbm_off + nbl * 16;                            // 4 bitmap words per box
+    list_off = wpre_off + nbl * 16;                           // outlier columns before each word
+    xo_off = list_off + kSmallListCap * 4;                    // X of the listed columns, fp16 [cap][16]
+    sc_off = xo_off + kSmallListCap * LT * 2;                 // SCB and bias of the tile's rows
+    xch_off = sc_off + 2 * LM * 4;
+    red_off = xch_off + (ks > 1 ? (LMAXKS * LT + LMAXKS) * 4 : 0);
+    misc_off = red_off + (ks > 1 ? 2 * LM * LT * 4 : 0);
     bar_off = (misc_off + 4 * LT * 4 + 32 + 7) & ~7;
     total = bar_off + (2 * LRS + 1) * 8 + 1024;  // + slack to align the ring to 1024 bytes
   }
@@ -80,17 +91,11 @@ __device__ __forceinline__ uint32_t small_code(float x, float r) {
   return q;
 }
 
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-
 }  // namespace
 
 size_t linear_small_smem(int K, int ks) {
   const int nbox = (K + 127) / 128;
-  return static_cast<size_t>(SmallLayout((nbox + ks - 1) / ks).total);
+  return static_cast<size_t>(SmallLayout((nbox + ks - 1) / ks, ks).total);
 }
 
 int linear_small_split(int N, int K, int num_sms) {
@@ -113,11 +118,17 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   const int kb0 = rank * nbox / KS, kb1 = (rank + 1) * nbox / KS;  // this CTA's boxes
   const int nbl = kb1 - kb0;
   const int nbl_max = (nbox + KS - 1) / KS;                         // the layout is the same in every CTA
-  const SmallLayout Lay(nbl_max);
+  const SmallLayout Lay(nbl_max, KS);
   uint8_t* ring = smem;
   uint8_t* ca = smem + Lay.ca_off;
   uint32_t* sbm = reinterpret_cast<uint32_t*>(smem + Lay.sbm_off);
+  int32_t* s_wpre = reinterpret_cast<int32_t*>(smem + Lay.wpre_off);
   int32_t* s_list = reinterpret_cast<int32_t*>(smem + Lay.list_off);
+  __half* xo = reinterpret_cast<__half*>(smem + Lay.xo_off);
+  float* s_sb = reinterpret_cast<float*>(smem + Lay.sc_off);
+  float* s_bv = s_sb + LM;
+  uint32_t* s_xmax = reinterpret_cast<uint32_t*>(smem + Lay.xch_off);  // [KS][16] row maxima of each CTA
+  uint32_t* s_xcnt = s_xmax + LMAXKS * LT;                               // [KS] outlier columns of each CTA
   int32_t* red_c = reinterpret_cast<int32_t*>(smem + Lay.red_off);
   float* red_d = reinterpret_cast<float*>(red_c + LM * LT);
   uint32_t* s_rowmax = reinterpret_cast<uint32_t*>(smem + Lay.misc_off);  // this slice's maxima (fp32 bits)
@@ -136,6 +147,29 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   const int RS = Lay.stages;
   const int nvec = (k1 - k0) >> 3, nwords = nbl * 4;
   const bool use_tau = tau > 0.f;
+
+  // the first X vectors and this tile's row scales and bias are requested before the set-up,
+  // which hides their latency
+  const int items = M * nvec;
+  const bool one_chunk = items <= LPU * LTHREADS;
+  uint4 xv[LPU];
+  auto load_x = [&](int base) {
+#pragma unroll
+    for (int u = 0; u < LPU; ++u) {
+      const int it = base + u * LTHREADS + tid;
+      xv[u] = make_uint4(0, 0, 0, 0);
+      if (it < items) {
+        const int r = it / nvec;
+        xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + k0) + (it - r * nvec));
+      }
+    }
+  };
+  load_x(0);
+  float sb_row = 0.f, bv_row = 0.f;
+  if (tid < LM && n0 + tid < N) {
+    sb_row = __ldg(SCB + n0 + tid);
+    if (bias != nullptr) bv_row = __half2float(bias[n0 + tid]);
+  }
 
   if (tid == 0) {
     for (int s = 0; s < LRS; ++s) {
@@ -160,6 +194,9 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
+  // first half of a cluster barrier: its wait (before the first store into another CTA's
+  // shared memory) guarantees that every CTA of the cluster has started
+  if (KS > 1) cluster_arrive_relaxed();
 
   // the weight slice does not depend on X: request the first stages now
   uint32_t filled = 0, fill_parity = 0;
@@ -178,19 +215,8 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   // Items (row, 8-column vector) in chunks of LPU per thread: all LPU loads of
   // a chunk are issued before any is used.  When the slice fits in one chunk it
   // stays in registers for the codes; otherwise they read each chunk again.
-  const int items = M * nvec;
-  const bool one_chunk = items <= LPU * LTHREADS;
-  uint4 xv[LPU];
   for (int base = 0; base < items; base += LPU * LTHREADS) {   // row maxima below the threshold, column flags
-#pragma unroll
-    for (int u = 0; u < LPU; ++u) {
-      const int it = base + u * LTHREADS + tid;
-      xv[u] = make_uint4(0, 0, 0, 0);
-      if (it < items) {
-        const int r = it / nvec;
-        xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + k0) + (it - r * nvec));
-      }
-    }
+    if (base > 0) load_x(base);
 #pragma unroll
     for (int u = 0; u < LPU; ++u) {   // (uniform trip count: whole warps vote below)
       const int it = base + u * LTHREADS + tid;
@@ -224,6 +250,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     }
   }
   __syncthreads();
+  if (KS > 1) cluster_wait();
   if (warp == 0) {   // this slice's sorted outlier list (ascending columns)
     const int per = (nwords + 31) / 32;
     const int w0 = min(lane * per, nwords), w1 = min(w0 + per, nwords);
@@ -237,6 +264,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     }
     int pos = incl - cnt;
     for (int w = w0; w < w1; ++w) {
+      s_wpre[w] = pos;
       uint32_t bits = sbm[w];
       while (bits) {
         const int b = __ffs(bits) - 1;
@@ -246,25 +274,36 @@ __global__ void __launch_bounds__(LTHREADS, 1)
       }
     }
     if (lane == 31) *s_cnt = incl;
+    // row maxima and the count go to every CTA of the cluster (this one included)
+    if (KS > 1) {
+      if (lane < LT) {
+        const uint32_t a = smem_addr(s_xmax + rank * LT + lane), m = s_rowmax[lane];
+        for (int r = 0; r < KS; ++r) st_cluster_u32(map_to_rank(a, r), m);
+      } else if (lane == 31) {
+        const uint32_t a = smem_addr(s_xcnt + rank);
+        for (int r = 0; r < KS; ++r) st_cluster_u32(map_to_rank(a, r), static_cast<uint32_t>(incl));
+      }
+    }
+  }
+  if (tid < LM) {
+    s_sb[tid] = sb_row;
+    s_bv[tid] = bv_row;
   }
   // ---------------------------------------------------------------- exchange with the cluster
   if (KS > 1) cluster_sync(); else __syncthreads();
+  // the pushed values are local now
   if (tid < LT) {
     uint32_t m = s_rowmax[tid];
-    if (KS > 1) {
-      const uint32_t a = smem_addr(s_rowmax + tid);
-      for (int r = 0; r < KS; ++r) m = max(m, ld_cluster_u32(map_to_rank(a, r)));
-    }
+    for (int r = 0; r < KS && KS > 1; ++r) m = max(m, s_xmax[r * LT + tid]);
     const float amax = tid < M ? __uint_as_float(m) : 0.f;
     s_r[tid] = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
     s_sa[tid] = amax * (1.0f / 16129.0f);
   } else if (tid == LT) {
     int before = 0, all = *s_cnt;
     if (KS > 1) {
-      const uint32_t a = smem_addr(s_cnt);
       all = 0;
       for (int r = 0; r < KS; ++r) {
-        const int c = static_cast<int>(ld_cluster_u32(map_to_rank(a, r)));
+        const int c = static_cast<int>(s_xcnt[r]);
         if (r < rank) before += c;
         all += c;
       }
@@ -274,16 +313,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   }
   __syncthreads();
   for (int base = 0; base < items; base += LPU * LTHREADS) {   // codes into the swizzled K-major tile
-    if (!one_chunk) {
-#pragma unroll
-      for (int u = 0; u < LPU; ++u) {
-        const int it = base + u * LTHREADS + tid;
-        if (it < items) {
-          const int r = it / nvec;
-          xv[u] = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + k0) + (it - r * nvec));
-        }
-      }
-    }
+    if (!one_chunk) load_x(base);
 #pragma unroll
     for (int u = 0; u < LPU; ++u) {
       const int it = base + u * LTHREADS + tid;
@@ -301,10 +331,16 @@ __global__ void __launch_bounds__(LTHREADS, 1)
         const uint32_t hi = __byte_perm(small_code(b.x, rs), small_code(b.y, rs), 0x0040);
         w[p] = __byte_perm(lo, hi, 0x5410);
       }
-      if (fl) {  // outlier columns carry code 0
+      if (fl) {  // outlier columns carry code 0; their X values go to xo at their list position
+        const __half* hx = reinterpret_cast<const __half*>(&xv[u]);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          if (fl & (1u << e)) w[e >> 2] &= ~(0xffu << ((e & 3) * 8));
+          if (fl & (1u << e)) {
+            w[e >> 2] &= ~(0xffu << ((e & 3) * 8));
+            const int c = 8 * v + e, wd = c >> 5;
+            const int pos = s_wpre[wd] + __popc(sbm[wd] & ((1u << (c & 31)) - 1u));
+            if (pos < kSmallListCap) xo[pos * LT + r] = hx[e];
+          }
       }
       // byte kk = 8v of row r in the slice: box kk / 128, 16-byte chunk q = (kk % 128) / 16 stored at q ^ (r % 8)
       const int kk = 8 * v, box = kk >> 7, q = (kk & 127) >> 4;
@@ -396,7 +432,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
             static_cast<float>(static_cast<int8_t>(sa[box * LBOX + row * 128 + (((b >> 4) ^ (row & 7)) << 4) + (b & 15)]));
 #pragma unroll
         for (int t = 0; t < LT; ++t)
-          if (t < M) d[t] = fmaf(__half2float(X[static_cast<size_t>(t) * K + j]), w, d[t]);
+          if (t < M) d[t] = fmaf(__half2float(xo[cur * LT + t]), w, d[t]);
         ++cur;
       }
       __syncwarp();
@@ -415,8 +451,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     if (KS == 1) {
       const int n = n0 + row;
       if (n < N) {
-        const float sb = __ldg(SCB + n);
-        const float bv = bias != nullptr ? __half2float(bias[n]) : 0.f;
+        const float sb = s_sb[row], bv = s_bv[row];
 #pragma unroll
         for (int t = 0; t < LT; ++t) {
           if (t >= M) break;
@@ -426,11 +461,15 @@ __global__ void __launch_bounds__(LTHREADS, 1)
         }
       }
     } else {
-      // partials of row `row`: 16 int32 and 16 fp32
+      // partials of row `row` (16 int32, 16 fp32) go to the CTA that finishes the row
+      const int rpr = LM / KS, owner = row / rpr, slot = row - owner * rpr;
+      const uint32_t ac = map_to_rank(smem_addr(red_c + (rank * rpr + slot) * LT), owner);
+      const uint32_t ad = map_to_rank(smem_addr(red_d + (rank * rpr + slot) * LT), owner);
 #pragma unroll
       for (int ch = 0; ch < LT / 4; ++ch) {
-        *reinterpret_cast<uint4*>(red_c + row * LT + 4 * ch) = make_uint4(c[4 * ch], c[4 * ch + 1], c[4 * ch + 2], c[4 * ch + 3]);
-        *reinterpret_cast<float4*>(red_d + row * LT + 4 * ch) = make_float4(d[4 * ch], d[4 * ch + 1], d[4 * ch + 2], d[4 * ch + 3]);
+        st_cluster_v4(ac + 16u * ch, c[4 * ch], c[4 * ch + 1], c[4 * ch + 2], c[4 * ch + 3]);
+        st_cluster_v4(ad + 16u * ch, __float_as_uint(d[4 * ch]), __float_as_uint(d[4 * ch + 1]),
+                      __float_as_uint(d[4 * ch + 2]), __float_as_uint(d[4 * ch + 3]));
       }
     }
   }
@@ -443,25 +482,21 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   }
   if (KS > 1) {
     // ---------------------------------------------------------------- sum of the cluster's partials
-    cluster_sync();
-    const int r0 = rank * LM / KS, r1 = (rank + 1) * LM / KS;
-    const uint32_t ac = smem_addr(red_c), ad = smem_addr(red_d);
-    for (int e = tid; e < (r1 - r0) * LT; e += LTHREADS) {
-      const int rl = r0 + e / LT, t = e % LT, n = n0 + rl;
+    cluster_sync();   // every partial of this CTA's rows has arrived; nothing is read remotely after this
+    const int rpr = LM / KS;
+    for (int e = tid; e < rpr * LT; e += LTHREADS) {
+      const int slot = e / LT, t = e % LT, rl = rank * rpr + slot, n = n0 + rl;
       if (t >= M || n >= N) continue;
       int32_t csum = 0;
       float dsum = 0.f;
-      const uint32_t off = 4u * static_cast<uint32_t>(rl * LT + t);
-      for (int r = 0; r < KS; ++r) {
-        csum += static_cast<int32_t>(ld_cluster_u32(map_to_rank(ac + off, r)));
-        dsum += __uint_as_float(ld_cluster_u32(map_to_rank(ad + off, r)));
+      for (int r = 0; r < KS; ++r) {   // rank order
+        csum += red_c[(r * rpr + slot) * LT + t];
+        dsum += red_d[(r * rpr + slot) * LT + t];
       }
-      const float sb = __ldg(SCB + n);
-      const float bv = bias != nullptr ? __half2float(bias[n]) : 0.f;
+      const float sb = s_sb[rl], bv = s_bv[rl];
       const float y = fmaf(dsum, sb * (1.0f / 127.0f), fmaf(static_cast<float>(csum), s_sa[t] * sb, bv));
       out[static_cast<size_t>(t) * N + n] = __float2half_rn(y);
     }
-    cluster_sync();   // this CTA's partials stay in place until every CTA has read them
   }
   tc_fence_before_sync();
   __syncthreads();
