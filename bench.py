@@ -463,10 +463,13 @@ def measure_other(i8, torch, dev, st, world, dist, reps: int = 50):
     # single linear: eager and graph-replayed
     L = W["C1"].layers[0]
     a = prepared("C1", 0, L)
-    us_eager = timed(lambda: run(L, *a))
+    dX, CB, SCB, db, out, _ = a
+    layer = i8.Linear8bitLt(CB, SCB, db, L.threshold, MAX_OUTLIER_COLS)
+    us_eager_fn = timed(lambda: run(L, *a))
+    us_eager = timed(lambda: layer(dX, out=out))
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        run(L, *a)
+        layer(dX, out=out)
     us_graph_1 = timed(graph.replay)
     del graph
     # a graph of GRAPH_CALLS forwards: the device time per forward once the host no longer
@@ -474,11 +477,14 @@ def measure_other(i8, torch, dev, st, world, dist, reps: int = 50):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for _ in range(GRAPH_CALLS):
-            run(L, *a)
+            layer(dX, out=out)
     us_graph = timed(graph.replay, n=max(1, reps // 5)) / GRAPH_CALLS
     del graph
-    res["single_linear"] = {"shape": f"{L.M}x{L.K}->{L.N}", "outlier_cols": status(a[5]),
+    res["single_linear"] = {"shape": f"{L.M}x{L.K}->{L.N}", "outlier_cols": status(layer.last_workspace),
                             "us_eager": round(us_eager, 2), "us_graph": round(us_graph, 2),
+                            "api": "Linear8bitLt layer (weights checked once); "
+                                   "us_eager_function: i8_linear8bit_forward with every argument checked",
+                            "us_eager_function": round(us_eager_fn, 2),
                             "us_graph_one_per_replay": round(us_graph_1, 2),
                             "graph_calls": GRAPH_CALLS,
                             "TOPS_eager": round(L.ops / us_eager / 1e6, 2),

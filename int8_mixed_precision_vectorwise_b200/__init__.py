@@ -34,3 +34,4 @@ from ._binding import (  # noqa: F401
     i8_selftest_bounded_wait,
     lib,
 )
+from .layer import Linear8bitLt  # noqa: F401

@@ -141,7 +141,8 @@ def _stream_handle(index):
 def _fits(t, dtype, shape, index):
     """True when t is a contiguous CUDA tensor of `dtype` and `shape` on device `index`
     (the cheap test of the per-call path; on False the detailed checks name the problem)."""
-    return (isinstance(t, torch.Tensor) and t.dtype is dtype and t.is_cuda and t.get_device() == index
+    # (get_device() is -1 for a CPU tensor, never a CUDA index)
+    return (isinstance(t, torch.Tensor) and t.dtype is dtype and t.get_device() == index
             and t.shape == shape and t.is_contiguous())
 
 

@@ -118,14 +118,39 @@ EncodeTiledFn encode_fn() {
 bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
                uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
                CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+  // A map is a function of these arguments alone (address, sizes, box, swizzle), so the
+  // last few encoded per host thread are kept and copied on a repeat: a layer called
+  // again with the same weight skips the encoder, a per-call host cost of the small forward.
+  struct Entry {
+    CUtensorMap map;
+    const void* base;
+    uint64_t inner, rows, stride;
+    uint32_t box_inner, box_rows;
+    int dt, swz;
+    bool valid;
+  };
+  static thread_local Entry cache[8];
+  static thread_local unsigned next = 0;
+  for (const Entry& e : cache)
+    if (e.valid && e.base == base && e.inner == inner && e.rows == rows && e.stride == row_stride_bytes &&
+        e.box_inner == box_inner && e.box_rows == box_rows && e.dt == static_cast<int>(dt) &&
+        e.swz == static_cast<int>(swz)) {
+      *tm = e.map;
+      return true;
+    }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {row_stride_bytes};
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  Entry& e = cache[next++ % 8];
+  e = Entry{*tm, base, inner, rows, row_stride_bytes, box_inner, box_rows, static_cast<int>(dt),
+            static_cast<int>(swz), true};
+  return true;
 }
 
 // SM count of the current device, cached per device (calls may come from

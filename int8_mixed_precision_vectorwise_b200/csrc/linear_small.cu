@@ -148,8 +148,45 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   const int nvec = (k1 - k0) >> 3, nwords = nbl * 4;
   const bool use_tau = tau > 0.f;
 
-  // the first X vectors and this tile's row scales and bias are requested before the set-up,
-  // which hides their latency
+  // ---------------------------------------------------------------- set-up (no global memory)
+  // The kernel is a programmatic dependent launch: this part may run while the previous
+  // kernel of the stream finishes; every global access comes after pdl_wait().
+  if (tid == 0) {
+    for (int s = 0; s < LRS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + 4);   // the MMAs' commit and the 4 outlier / epilogue warps
+    }
+    mbar_init(acc_full, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, LTMEM_COLS);
+    tmem_relinquish();
+  }
+  for (int w = tid; w < nwords; w += LTHREADS) sbm[w] = 0u;
+  if (tid < LT) s_rowmax[tid] = 0u;
+  {  // zero the code tile: rows past M and bytes past K must be 0 for the MMA
+    uint4* z = reinterpret_cast<uint4*>(ca);
+    for (int i = tid; i < nbl * LCA_BOX / 16; i += LTHREADS) z[i] = make_uint4(0, 0, 0, 0);
+  }
+  pdl_wait();
+  pdl_launch_dependents();   // the next kernel's set-up may overlap the rest of this one
+
+  // the weight slice does not depend on X: thread 0 requests the first stages (its barriers
+  // are initialised and fenced above); then every thread requests its first X vectors and
+  // this tile's row scales and bias, whose latency the block barrier below overlaps
+  uint32_t filled = 0, fill_parity = 0;
+  if (tid == 0) {
+    for (int st = 0; st < nstage && st < RS; ++st) {
+      const int b0 = st * LSB, nb = min(LSB, nbl - b0);
+      mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nb * LBOX));
+      filled |= 1u << st;
+      for (int b = 0; b < nb; ++b)
+        tma_load_2d(ring + st * LSTAGE + b * LBOX, &tmW, &full[st], (kb0 + b0 + b) * 128, n0);
+    }
+  }
   const int items = M * nvec;
   const bool one_chunk = items <= LPU * LTHREADS;
   uint4 xv[LPU];
@@ -170,26 +207,6 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     sb_row = __ldg(SCB + n0 + tid);
     if (bias != nullptr) bv_row = __half2float(bias[n0 + tid]);
   }
-
-  if (tid == 0) {
-    for (int s = 0; s < LRS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);   // the MMAs' commit and the 4 outlier / epilogue warps
-    }
-    mbar_init(acc_full, 1);
-    *s_abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(s_tmem, LTMEM_COLS);
-    tmem_relinquish();
-  }
-  for (int w = tid; w < nwords; w += LTHREADS) sbm[w] = 0u;
-  if (tid < LT) s_rowmax[tid] = 0u;
-  {  // zero the code tile: rows past M and bytes past K must be 0 for the MMA
-    uint4* z = reinterpret_cast<uint4*>(ca);
-    for (int i = tid; i < nbl * LCA_BOX / 16; i += LTHREADS) z[i] = make_uint4(0, 0, 0, 0);
-  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -197,19 +214,6 @@ __global__ void __launch_bounds__(LTHREADS, 1)
   // first half of a cluster barrier: its wait (before the first store into another CTA's
   // shared memory) guarantees that every CTA of the cluster has started
   if (KS > 1) cluster_arrive_relaxed();
-
-  // the weight slice does not depend on X: request the first stages now
-  uint32_t filled = 0, fill_parity = 0;
-  if (tid == 0) {
-    tma_prefetch_desc(&tmW);
-    for (int st = 0; st < nstage && st < RS; ++st) {
-      const int b0 = st * LSB, nb = min(LSB, nbl - b0);
-      mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(nb * LBOX));
-      filled |= 1u << st;
-      for (int b = 0; b < nb; ++b)
-        tma_load_2d(ring + st * LSTAGE + b * LBOX, &tmW, &full[st], (kb0 + b0 + b) * 128, n0);
-    }
-  }
 
   // ---------------------------------------------------------------- this slice of X (all threads)
   // Items (row, 8-column vector) in chunks of LPU per thread: all LPU loads of
@@ -526,13 +530,15 @@ cudaError_t launch_linear_small(const CUtensorMap& tmW, const __half* X, int M, 
   cfg.blockDim = dim3(LTHREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = ks;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = ks;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = ks > 1 ? 1 : 0;
+  cfg.numAttrs = ks > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_linear_small, tmW, X, M, N, K, tau, cap, SCB, bias, out, hdr, limit_ns,
                             reset_status ? 1 : 0, ks);
 }

@@ -135,3 +135,28 @@ def test_other_ops(fake):
     assert dX.shape == (M, K)
     with pytest.raises(ValueError, match="shape"):
         b.i8_linear8bit_backward_input(z((M, N), torch.float16), Wt, dX=z((M, K + 1), torch.float16))
+
+
+def test_layer_checks_weights_once_and_x_per_call(fake):
+    from int8_mixed_precision_vectorwise_b200.layer import Linear8bitLt
+    N, K = 24, 32
+    CB, SCB, bias = z((N, K), torch.int8), z(N, torch.float32), z(N, torch.float16)
+    layer = Linear8bitLt(CB, SCB, bias, threshold=6.0)
+    out = layer(z((5, K), torch.float16))
+    assert out.shape == (5, N) and out.dtype == torch.float16
+    name, args = fake.calls[-1]
+    assert name == "i8_linear8bit_forward" and args[4:8] == (5, N, K, 6.0)
+    assert args[1] == CB.data_ptr() and args[3] == bias.data_ptr()
+    ws5 = layer.workspace(5)
+    buf = z((3, N), torch.float16)
+    assert layer(z((3, K), torch.float16), out=buf) is buf       # a caller buffer is used as given
+    layer(z((5, K), torch.float16))
+    assert layer.workspace(5) is ws5                             # one workspace per token count
+    with pytest.raises(ValueError, match="shape"):
+        layer(z((5, K + 16), torch.float16))
+    with pytest.raises(TypeError):
+        layer(z((5, K), torch.float32))
+    with pytest.raises(ValueError, match="shape"):
+        layer(z((5, K), torch.float16), out=z((5, N + 8), torch.float16))
+    with pytest.raises(ValueError, match="shape"):
+        Linear8bitLt(CB, z(N + 1, torch.float32))

@@ -510,3 +510,21 @@ def test_forward_multi_reuses_workspace(i8):
             for g in range(len(Ns)):
                 rCB, rSCB = oracle.quantize_weight_rowwise(W[g])
                 assert_close(host(outs[g]), oracle.linear8bit_forward(X, rCB, rSCB, None, 6.0), f"reuse {M} {g}")
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 1024, 1024), (3, 300, 272), (300, 520, 1040)])
+def test_layer_matches_function(i8, M, N, K):
+    """Linear8bitLt (weights checked once, a workspace per token count) gives the function's
+    output bit for bit, call after call, and the oracle's within tolerance."""
+    X, _ = act(M, K, 3, mag=(8.0, 60.0), seed=61 + M)
+    W = wl.weight(62 + N, N, K)
+    b = wl.bias(63, N)
+    rCB, rSCB = oracle.quantize_weight_rowwise(W)
+    dCB, dSCB, db = dev(rCB), dev(rSCB), dev(b)
+    layer = i8.Linear8bitLt(dCB, dSCB, db, 6.0)
+    ref_out, ws = i8.i8_linear8bit_forward(dev(X), dCB, dSCB, db, 6.0)
+    for _ in range(2):
+        o = layer(dev(X))
+        assert torch.equal(o, ref_out)
+        assert i8.i8_read_status(layer.last_workspace) == i8.i8_read_status(ws)
+    assert_close(host(o), oracle.linear8bit_forward(X, rCB, rSCB, b, 6.0), "layer")
