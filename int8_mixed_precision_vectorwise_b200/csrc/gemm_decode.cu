@@ -41,6 +41,7 @@ namespace {
 constexpr int DM = 128;                    // weight rows per tile (MMA M)
 constexpr int DT = kDecodeMaxTokens;       // token columns (MMA N), zero padded
 constexpr int DK = 128;                    // bytes of K per swizzle atom / TMA box
+constexpr int DL2_AHEAD = 8;               // weight stages past the ring prefetched into L2 before the wait
 constexpr int DTHREADS = 64 + 128 + 32;
 constexpr int DA_BYTES = DM * DK;          // 16 KB of weights per box
 constexpr int DB_BYTES = DT * DK;          // 2 KB of codes per box
@@ -163,6 +164,13 @@ __global__ void __launch_bounds__(DTHREADS, 1)
 #pragma unroll
         for (int c = 0; c < C; ++c)
           tma_load_2d(smem + i * DSTAGE_BYTES + c * DA_BYTES, &tmW, &full[i], k * DKS + c * DK, tile * DM);
+      }
+      // the weight stages after the ring go to L2 while the preceding kernel finishes, so
+      // HBM keeps streaming during the wait and those stages later load from L2
+      for (int i = npre; i < min(npos, npre + DL2_AHEAD); ++i) {
+        const int pos = start + i, tile = pos / kb, k = pos - tile * kb;
+#pragma unroll
+        for (int c = 0; c < C; ++c) tma_prefetch_l2_2d(&tmW, k * DKS + c * DK, tile * DM);
       }
       pdl_wait();
       for (int i = 0; i < npre; ++i) {

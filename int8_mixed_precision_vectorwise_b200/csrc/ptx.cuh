@@ -109,6 +109,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* t
 
 // 1-D bulk copy global -> this CTA's shared memory, completing `bytes` on
 // `bar`.  Addresses 16-byte aligned, size a multiple of 16.
+// Bring a tile of a tensor into L2 (no shared-memory destination, no completion
+// signal): a hint that lets HBM stream ahead while the consumer cannot yet take data.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* tm, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
