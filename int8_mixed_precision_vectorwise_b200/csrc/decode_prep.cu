@@ -5,7 +5,8 @@
 // Part 1", section "Improved kernels for inference", int8_vectorwise_quant;
 // the mixed decomposition of "`bitsandbytes` - `Linear8bitLt` integration
 // into `transformers` models", section "About the mixed quantization method
-// in few words") -- runs on one cluster of 8 CTAs.
+// in few words") -- runs on one cluster of 8 CTAs (16 for long rows of many
+// tokens, M * K >= kDecodeHeavyPrep, when the device can place such a cluster).
 //
 // Each CTA owns a contiguous range of columns for all rows.  A column is an
 // outlier column when any of its (at most 16) elements reaches the threshold,
@@ -18,10 +19,12 @@
 //   pass 1  X -> per-row max |x| over elements below the threshold (packed
 //           fp16 max; per-element test only where a vector reaches the
 //           threshold) and the CTA's outlier column flags
-//   sync    cluster barrier; row maxima and counts read from all 8 CTAs
+//   sync    cluster barrier; row maxima and counts read from all CTAs of the cluster
 //   pass 2  X (now in L2) -> codes (0 in outlier columns), SCA; the CTA's
 //           outlier columns go to idx / X_O at the offset of the CTAs before it
 #include <cuda_fp16.h>
+
+#include <atomic>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -30,7 +33,6 @@ namespace i8lt {
 
 namespace {
 
-constexpr int PC = kDecodePrepCluster;   // CTAs in the cluster
 constexpr int PT = 1024;                 // threads per CTA
 constexpr unsigned kAll = 0xffffffffu;
 constexpr int PU = 8;                    // X vectors per thread in flight
@@ -50,7 +52,9 @@ __device__ __forceinline__ uint32_t code_s8p(float x, float r) {
 
 }  // namespace
 
-__global__ void __cluster_dims__(kDecodePrepCluster, 1, 1) __launch_bounds__(1024, 1)
+// PC: CTAs in the cluster (the launch gives the cluster shape)
+template <int PC>
+__global__ void __launch_bounds__(1024, 1)
     k_decode_prep(const __half* __restrict__ X, int M, int K, float tau, int cap, int8_t* __restrict__ CA,
                   float* __restrict__ SCA, int32_t* __restrict__ idx, __half* __restrict__ XO, int ld_o,
                   uint32_t* __restrict__ hdr, int32_t* __restrict__ counters, int n_counters) {
@@ -262,9 +266,42 @@ __global__ void __cluster_dims__(kDecodePrepCluster, 1, 1) __launch_bounds__(102
   cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
 
-cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA,
-                               int32_t* idx, __half* XO, int ld_o, uint32_t* hdr, int32_t* counters, int n_counters,
-                               cudaStream_t st) {
+namespace {
+
+// Whether a cluster of kDecodePrepClusterBig CTAs of this kernel fits the device (a
+// non-portable size: it needs 16 SMs of one GPC); checked once per device.
+bool big_cluster_ok() {
+  static std::atomic<int> state[64];   // 0 unknown, 1 yes, 2 no
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const int st = state[dev].load(std::memory_order_acquire);
+  if (st != 0) return st == 1;
+  bool ok = cudaFuncSetAttribute(k_decode_prep<kDecodePrepClusterBig>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kDecodePrepClusterBig, 1, 1);
+    cfg.blockDim = dim3(PT, 1, 1);
+    cfg.dynamicSmemBytes = 4096;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = kDecodePrepClusterBig;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    ok = cudaOccupancyMaxActiveClusters(&clusters, k_decode_prep<kDecodePrepClusterBig>, &cfg) == cudaSuccess &&
+         clusters >= 1;
+  }
+  cudaGetLastError();   // a refused query leaves no error behind
+  state[dev].store(ok ? 1 : 2, std::memory_order_release);
+  return ok;
+}
+
+template <int PC>
+cudaError_t launch_prep_t(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA, int32_t* idx,
+                          __half* XO, int ld_o, uint32_t* hdr, int32_t* counters, int n_counters, cudaStream_t st) {
   const int span = ((K + PC - 1) / PC + 31) & ~31;
   const size_t smem = static_cast<size_t>((span + 31) / 32) * 4;
   cudaLaunchConfig_t cfg = {};
@@ -272,13 +309,33 @@ cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap
   cfg.blockDim = dim3(PT, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_decode_prep, X, M, K, tau, cap, CA, SCA, idx, XO, ld_o, hdr, counters,
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = PC;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k_decode_prep<PC>, X, M, K, tau, cap, CA, SCA, idx, XO, ld_o, hdr, counters,
                             n_counters);
+}
+
+}  // namespace
+
+int decode_prep_cluster(int M, int K) {
+  return static_cast<long long>(M) * K >= kDecodeHeavyPrep && big_cluster_ok() ? kDecodePrepClusterBig
+                                                                               : kDecodePrepCluster;
+}
+
+cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA,
+                               int32_t* idx, __half* XO, int ld_o, uint32_t* hdr, int32_t* counters, int n_counters,
+                               cudaStream_t st) {
+  if (decode_prep_cluster(M, K) == kDecodePrepClusterBig)
+    return launch_prep_t<kDecodePrepClusterBig>(X, M, K, tau, cap, CA, SCA, idx, XO, ld_o, hdr, counters, n_counters,
+                                                st);
+  return launch_prep_t<kDecodePrepCluster>(X, M, K, tau, cap, CA, SCA, idx, XO, ld_o, hdr, counters, n_counters, st);
 }
 
 }  // namespace i8lt

@@ -244,15 +244,15 @@ i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, in
 // Few-token GEMM: 128-byte K boxes per pipeline stage (512 bytes of each
 // weight row per stage) and the grid of the stream-K split (one CTA per SM, at
 // most kDecodeMaxGrid, never more CTAs than (tile, stage) work items).
-// `prep_elems` is the M*K the preparation kernel before it quantises: when it
-// is large, that kernel's cluster keeps its SMs busy for several microseconds
-// while the GEMM's CTAs would wait for them with an equal share of the weight
-// stream, so the GEMM leaves those SMs out.
+// `M_prep` is the number of rows the preparation kernel before it quantises (0:
+// none): when M_prep * K is large, that kernel's cluster keeps its SMs busy for
+// several microseconds while the GEMM's CTAs would wait for them with an equal
+// share of the weight stream, so the GEMM leaves those SMs out.
 constexpr int kDecodeBoxes = 4;
-constexpr long long kDecodeHeavyPrep = 16LL * 16384;
-int decode_grid(int N, int K, int sms, long long prep_elems) {
+int decode_grid(int N, int K, int sms, int M_prep) {
   const int total = ((N + 127) / 128) * ((K + 128 * kDecodeBoxes - 1) / (128 * kDecodeBoxes));
-  if (prep_elems >= kDecodeHeavyPrep) sms -= i8lt::kDecodePrepCluster;
+  if (M_prep > 0 && static_cast<long long>(M_prep) * K >= i8lt::kDecodeHeavyPrep)
+    sms -= i8lt::decode_prep_cluster(M_prep, K);
   int grid = sms < i8lt::kDecodeMaxGrid ? sms : i8lt::kDecodeMaxGrid;
   return grid > total ? total : grid;
 }
@@ -364,7 +364,7 @@ i8_status enqueue_gemm(const int8_t* CB, const float* SCB, const i8_half* bias, 
       return I8_ERR_CUDA;
     const int sms = num_sms();
     if (sms <= 0) return I8_ERR_CUDA;
-    return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms, static_cast<long long>(M) * K),
+    return cuda_status(i8lt::launch_gemm_decode(tmW, tmC, d, decode_grid(N, K, sms, M),
                                                 kDecodeBoxes, true, st));
   }
   GemmArgs a{};

@@ -115,11 +115,15 @@ inline int decode_slots(int N, int K) {
 cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
                                int boxes_per_stage, bool pdl, cudaStream_t st);
 
-// Few-token preparation on one cluster of kDecodePrepCluster CTAs (M <= 16):
+// Few-token preparation on one cluster of decode_prep_cluster(M, K) CTAs (M <= 16):
 // codes, SCA, outlier list, X_O (zero padded to a multiple of 16 columns), the
 // header words (status, used, total) and zeroed split-K counters, all in one
-// launch.  XO may be null when cap == 0.
+// launch.  XO may be null when cap == 0.  Clusters of 8 CTAs, or 16 (a
+// non-portable size) when M * K >= kDecodeHeavyPrep and the device can place one.
 constexpr int kDecodePrepCluster = 8;
+constexpr int kDecodePrepClusterBig = 16;
+constexpr long long kDecodeHeavyPrep = 16LL * 16384;
+int decode_prep_cluster(int M, int K);
 cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA,
                                int32_t* idx, __half* XO, int ld_o, uint32_t* hdr, int32_t* counters, int n_counters,
                                cudaStream_t st);

@@ -140,6 +140,8 @@ PREP_CASES = [
     (16, 1024, 8192, 8, 6.0, 256),     # few tokens
     (1, 4096, 28672, 3, 6.0, 256),
     (4, 2048, 4096, 40, 6.0, 256),     # few tokens, outliers in every CTA's column range
+    (16, 512, 28672, 40, 6.0, 256),    # few tokens on long rows: the 16-CTA preparation cluster
+    (12, 256, 24576, 10, 6.0, 64),     # the same, 12 tokens, ragged column ranges
     (300, 520, 1040, 80, 6.0, 101),    # 80 columns, a capacity that is not a multiple of 4
     (260, 300, 8192, 100, 6.0, 256),   # 100 columns on long rows
 ]
