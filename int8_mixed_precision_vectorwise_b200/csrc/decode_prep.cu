@@ -5,8 +5,8 @@
 // Part 1", section "Improved kernels for inference", int8_vectorwise_quant;
 // the mixed decomposition of "`bitsandbytes` - `Linear8bitLt` integration
 // into `transformers` models", section "About the mixed quantization method
-// in few words") -- runs on one cluster of 8 CTAs (16 for long rows of many
-// tokens, M * K >= kDecodeHeavyPrep, when the device can place such a cluster).
+// in few words") -- runs on one cluster of 8 CTAs (16 for long rows of several
+// tokens, when the device can place such a cluster).
 //
 // Each CTA owns a contiguous range of columns for all rows.  A column is an
 // outlier column when any of its (at most 16) elements reaches the threshold,
@@ -325,8 +325,9 @@ cudaError_t launch_prep_t(const __half* X, int M, int K, float tau, int cap, int
 }  // namespace
 
 int decode_prep_cluster(int M, int K) {
-  return static_cast<long long>(M) * K >= kDecodeHeavyPrep && big_cluster_ok() ? kDecodePrepClusterBig
-                                                                               : kDecodePrepCluster;
+  return K >= kDecodeLongRow && static_cast<long long>(M) * K >= kDecodeBigPrep && big_cluster_ok()
+             ? kDecodePrepClusterBig
+             : kDecodePrepCluster;
 }
 
 cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA,

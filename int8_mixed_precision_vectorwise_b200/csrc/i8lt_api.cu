@@ -251,8 +251,10 @@ i8_status run_gemm_f16(const __half* Aop, const __half* Bop, int M, int Nout, in
 constexpr int kDecodeBoxes = 4;
 int decode_grid(int N, int K, int sms, int M_prep) {
   const int total = ((N + 127) / 128) * ((K + 128 * kDecodeBoxes - 1) / (128 * kDecodeBoxes));
-  if (M_prep > 0 && static_cast<long long>(M_prep) * K >= i8lt::kDecodeHeavyPrep)
-    sms -= i8lt::decode_prep_cluster(M_prep, K);
+  if (M_prep > 0) {
+    const int pc = i8lt::decode_prep_cluster(M_prep, K);
+    if (pc == i8lt::kDecodePrepClusterBig || static_cast<long long>(M_prep) * K >= i8lt::kDecodeHeavyPrep) sms -= pc;
+  }
   int grid = sms < i8lt::kDecodeMaxGrid ? sms : i8lt::kDecodeMaxGrid;
   return grid > total ? total : grid;
 }

@@ -119,9 +119,14 @@ cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmC, c
 // codes, SCA, outlier list, X_O (zero padded to a multiple of 16 columns), the
 // header words (status, used, total) and zeroed split-K counters, all in one
 // launch.  XO may be null when cap == 0.  Clusters of 8 CTAs, or 16 (a
-// non-portable size) when M * K >= kDecodeHeavyPrep and the device can place one.
+// non-portable size) for long rows of several tokens (K >= kDecodeLongRow and
+// M * K >= kDecodeBigPrep) when the device can place one.
 constexpr int kDecodePrepCluster = 8;
 constexpr int kDecodePrepClusterBig = 16;
+constexpr int kDecodeLongRow = 16384;
+constexpr long long kDecodeBigPrep = 4LL * 16384;
+// A preparation this large keeps its SMs busy long enough that the GEMM after it
+// leaves them out of its grid (so does a 16-CTA preparation).
 constexpr long long kDecodeHeavyPrep = 16LL * 16384;
 int decode_prep_cluster(int M, int K);
 cudaError_t launch_decode_prep(const __half* X, int M, int K, float tau, int cap, int8_t* CA, float* SCA,

@@ -142,6 +142,7 @@ PREP_CASES = [
     (4, 2048, 4096, 40, 6.0, 256),     # few tokens, outliers in every CTA's column range
     (16, 512, 28672, 40, 6.0, 256),    # few tokens on long rows: the 16-CTA preparation cluster
     (12, 256, 24576, 10, 6.0, 64),     # the same, 12 tokens, ragged column ranges
+    (4, 256, 28672, 5, 6.0, 64),       # 4 tokens on long rows: also the 16-CTA cluster
     (300, 520, 1040, 80, 6.0, 101),    # 80 columns, a capacity that is not a multiple of 4
     (260, 300, 8192, 100, 6.0, 256),   # 100 columns on long rows
 ]
