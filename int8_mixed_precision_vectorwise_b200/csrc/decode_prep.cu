@@ -27,6 +27,7 @@
 #include <atomic>
 
 #include "kernels.cuh"
+#include "per_device.h"
 #include "ptx.cuh"
 
 namespace i8lt {
@@ -271,32 +272,31 @@ namespace {
 // Whether a cluster of kDecodePrepClusterBig CTAs of this kernel fits the device (a
 // non-portable size: it needs 16 SMs of one GPC); checked once per device.
 bool big_cluster_ok() {
-  static std::atomic<int> state[64];   // 0 unknown, 1 yes, 2 no
+  static PerDeviceInt state;   // 1 yes, 2 no
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  const int st = state[dev].load(std::memory_order_acquire);
-  if (st != 0) return st == 1;
-  bool ok = cudaFuncSetAttribute(k_decode_prep<kDecodePrepClusterBig>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
-  if (ok) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kDecodePrepClusterBig, 1, 1);
-    cfg.blockDim = dim3(PT, 1, 1);
-    cfg.dynamicSmemBytes = 4096;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = kDecodePrepClusterBig;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    ok = cudaOccupancyMaxActiveClusters(&clusters, k_decode_prep<kDecodePrepClusterBig>, &cfg) == cudaSuccess &&
-         clusters >= 1;
-  }
-  cudaGetLastError();   // a refused query leaves no error behind
-  state[dev].store(ok ? 1 : 2, std::memory_order_release);
-  return ok;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  return state.get(dev, [] {
+    bool ok = cudaFuncSetAttribute(k_decode_prep<kDecodePrepClusterBig>,
+                                   cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    if (ok) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kDecodePrepClusterBig, 1, 1);
+      cfg.blockDim = dim3(PT, 1, 1);
+      cfg.dynamicSmemBytes = 4096;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = kDecodePrepClusterBig;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      ok = cudaOccupancyMaxActiveClusters(&clusters, k_decode_prep<kDecodePrepClusterBig>, &cfg) == cudaSuccess &&
+           clusters >= 1;
+    }
+    cudaGetLastError();   // a refused query leaves no error behind
+    return ok ? 1 : 2;
+  }) == 1;
 }
 
 template <int PC>

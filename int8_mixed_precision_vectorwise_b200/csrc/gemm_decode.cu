@@ -32,6 +32,7 @@
 #include <atomic>
 
 #include "kernels.cuh"
+#include "per_device.h"
 #include "ptx.cuh"
 
 namespace i8lt {
@@ -455,15 +456,16 @@ template <int C>
 static cudaError_t launch_decode_c(const CUtensorMap& tmW, const CUtensorMap& tmC, const DecodeArgs& a, int grid,
                                    bool pdl, cudaStream_t st) {
   // the shared-memory opt-in, once per device (calls may come from several host threads)
-  static std::atomic<bool> attr_done[64];
+  static PerDeviceOnce attr_done;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_i8_decode<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DecodeCfg<C>::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
-  }
+  cudaError_t e = cudaSuccess;
+  if (!attr_done.run(dev, [&] {
+        e = cudaFuncSetAttribute(k_gemm_i8_decode<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DecodeCfg<C>::SMEM_ALLOC);
+        return e == cudaSuccess;
+      }))
+    return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(DTHREADS, 1, 1);

@@ -48,6 +48,7 @@
 #include <type_traits>
 
 #include "kernels.cuh"
+#include "per_device.h"
 #include "ptx.cuh"
 
 namespace i8lt {
@@ -647,33 +648,29 @@ static GemmKernel gemm_kernel(GemmMode mode) {
 // Number of CTA pairs that fit on the device at once (cached per mode and
 // device; calls may come from several host threads, so the cache is atomic).
 static int max_pairs(GemmMode mode, int num_sms) {
-  static std::atomic<int> cache[3][64];
+  static PerDeviceInt cache[3];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
-  const int m = static_cast<int>(mode);
-  if (dev >= 0 && dev < 64) {
-    const int c = cache[m][dev].load(std::memory_order_relaxed);
-    if (c > 0) return c;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1), 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_ALLOC;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = 2;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel(mode), &cfg);
-  if (e != cudaSuccess || n <= 0) {
-    cudaGetLastError();
-    n = num_sms / 2;
-  }
-  if (dev >= 0 && dev < 64) cache[m][dev].store(n, std::memory_order_relaxed);
-  return n;
+  return cache[static_cast<int>(mode)].get(dev, [mode, num_sms] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1), 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_ALLOC;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel(mode), &cfg);
+    if (e != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms / 2;
+    }
+    return n;
+  });
 }
 
 cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, GemmMode mode, int num_sms, cudaStream_t st) {
@@ -681,15 +678,15 @@ cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& a, GemmMode mode, 
   // the shared-memory opt-in is a per-device property of the kernel: done once
   // per mode and device (several host threads may get here at once; setting it
   // twice is harmless)
-  static std::atomic<bool> attr_done[3][64];
-  const int m = static_cast<int>(mode);
+  static PerDeviceOnce attr_done[3];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev < 0 || dev >= 64 || !attr_done[m][dev].load(std::memory_order_acquire)) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel(mode), cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_done[m][dev].store(true, std::memory_order_release);
-  }
+  cudaError_t e = cudaSuccess;
+  if (!attr_done[static_cast<int>(mode)].run(dev, [&] {
+        e = cudaFuncSetAttribute(gemm_kernel(mode), cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+        return e == cudaSuccess;
+      }))
+    return e;
   const int tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
   const int pairs_fit = max_pairs(mode, num_sms);
   // fewer tiles than pairs: run each tile as two half tiles where that fits

@@ -14,6 +14,7 @@
 
 #include "../../include/i8lt.h"
 #include "kernels.cuh"
+#include "per_device.h"
 
 namespace {
 
@@ -156,17 +157,13 @@ bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64
 // SM count of the current device, cached per device (calls may come from
 // several host threads at once).
 int num_sms() {
-  static std::atomic<int> cache[64];
+  static i8lt::PerDeviceInt cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64) {
-    const int c = cache[dev].load(std::memory_order_relaxed);
-    if (c > 0) return c;
-  }
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
-  return n;
+  return cache.get(dev, [dev] {
+    int n = 0;
+    return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : 0;
+  });
 }
 
 inline i8_status cuda_status(cudaError_t e) { return e == cudaSuccess ? I8_OK : I8_ERR_CUDA; }

@@ -45,6 +45,7 @@
 #include <atomic>
 
 #include "kernels.cuh"
+#include "per_device.h"
 #include "ptx.cuh"
 
 namespace i8lt {
@@ -515,15 +516,16 @@ cudaError_t launch_linear_small(const CUtensorMap& tmW, const __half* X, int M, 
                                 bool reset_status, int num_sms, cudaStream_t st) {
   const int ks = linear_small_split(N, K, num_sms);
   const size_t smem = linear_small_smem(K, ks);
-  static std::atomic<bool> attr_done[64];
+  static PerDeviceOnce attr_done;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
-    cudaError_t e = cudaFuncSetAttribute(k_linear_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(linear_small_smem(kSmallMaxK, 1)));
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
-  }
+  cudaError_t e = cudaSuccess;
+  if (!attr_done.run(dev, [&] {
+        e = cudaFuncSetAttribute(k_linear_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(linear_small_smem(kSmallMaxK, 1)));
+        return e == cudaSuccess;
+      }))
+    return e;
   const int ntile = (N + LM - 1) / LM;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ntile * ks);
