@@ -63,6 +63,12 @@ QSHAPES = [
     (1, 16, 0.0, 0), (3, 1024, 6.0, 2), (37, 4096, 6.0, 4), (130, 5120, 6.0, 5), (64, 8192, 6.0, 8),
     (16, 11008, 6.0, 11), (5, 28672, 6.0, 8), (3, 40000, 6.0, 3), (300, 2064, 0.0, 0), (1000, 272, 6.0, 1),
     (9, 4096, 6.0, 0), (257, 1040, 2.5, 0),
+    # enough rows for the ring-fed kernel (one CTA per SM, rows bulk-copied into shared memory)
+    (4099, 4096, 6.0, 9),     # 2 rows per stage, an odd number of rows
+    (2500, 1040, 6.0, 3),     # 2 rows per stage, short rows
+    (1300, 8192, 6.0, 12),    # 1 row per stage
+    (700, 11008, 0.0, 0),     # 6 vectors per thread, threshold 0
+    (600, 16384, 6.0, 5),     # 8 vectors per thread, 4 stages
 ]
 
 
