@@ -196,6 +196,28 @@ def decode_bytes(L) -> int:
     return L.N * L.K + 4 * L.N + 2 * L.M * L.K + 2 * L.M * L.N
 
 
+def graph_us(torch, dev, st, fn, calls: int, replays: int = 3) -> float:
+    """Device time per call of `fn` with the host out of the way: `calls` calls captured in one
+    CUDA graph, replayed `replays` times between CUDA events on `st` after one warm-up replay.
+    A call whose host side (argument checks, the C entry, the launches) takes longer than its
+    kernels leaves the GPU idle between back-to-back eager calls; the replay does not."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(calls):
+            fn()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(replays):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) / (replays * calls) * 1e3
+    del g
+    return us
+
+
 def measure_decode(i8, torch, dev, st, world, dist, reps: int = 20):
     """Every point of the decode grid (tokens {1, 4, 16} x outlier columns {0, 1, 8}) on both
     Llama-70B FFN shapes.  Weights (235 MB each, > L2) stream from HBM every call.  Per point:
@@ -243,6 +265,7 @@ def measure_decode(i8, torch, dev, st, world, dist, reps: int = 20):
                 i8.i8_linear8bit_matmul_dequant(CB, SCB, None, L.M, L.threshold, out, ws, MAX_OUTLIER_COLS)
                 ev[r][2].record(st)
             torch.cuda.synchronize(dev)
+            us_graph = graph_us(torch, dev, st, fwd, reps)
             code, _ = i8.i8_read_status(ws)
             if code != 0:
                 raise RuntimeError(f"decode status {i8.STATUS.get(code, code)}")
@@ -252,11 +275,15 @@ def measure_decode(i8, torch, dev, st, world, dist, reps: int = 20):
             gbs = decode_bytes(L) / us / 1e3
             points.append({"shape": f"{L.M}x{L.K}->{L.N}", "tokens": L.M, "outlier_cols": L.n_out,
                            "us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                           "us_graph": round(us_graph, 2),
+                           "frac_graph": round(decode_bytes(L) / us_graph / 1e3 / hbm, 4),
                            "prep_alone_us": round(prep_us, 2), "gemm_alone_us": round(gemm_us, 2),
                            "gemm_alone_frac": round(decode_bytes(L) / gemm_us / 1e3 / hbm, 4)})
     best = max(points, key=lambda q: q["GB/s"])
     worst = min(points, key=lambda q: q["GB/s"])
     return {"metric": "decode weight-read GB/s (whole forward per call)", "peak_gbs": hbm,
+            "timing": f"us: CUDA events over {reps} back-to-back eager calls; us_graph: the same calls "
+                      "replayed from a CUDA graph (no host time between forwards)",
             "peak_source": "of measured hbm_gbs" if measured_peaks() else "of fallback",
             "bytes": "N*K + 4N + 2MK + 2MN per call", "points": points,
             "best_GB/s": best["GB/s"], "best_frac": best["frac"],
@@ -293,16 +320,32 @@ def measure_quant(i8, torch, dev, st, world, dist, reps: int = 40):
             e1.record(st)
             torch.cuda.synchronize(dev)
             us = e0.elapsed_time(e1) / reps * 1e3
-            gbs = (2 * M * K + M * K + 4 * M + K / 8) / us / 1e3
-            tag = "kernel" if tau == 0.0 else "op_tau6"
-            row.update({f"{tag}_us": round(us, 2), f"{tag}_GB/s": round(gbs, 1), f"{tag}_frac": round(gbs / hbm, 4)})
+            byts = 2 * M * K + M * K + 4 * M + K / 8
+            gbs = byts / us / 1e3
+            if tau == 0.0:
+                # the kernel alone: the calls replayed from a graph (an eager call's host side
+                # takes longer than this kernel)
+                order = iter(range(reps))
+
+                def one():  # the next input of the rotation
+                    r = next(order)
+                    i8.i8_quantize_rowwise(Xs[r % n], tau, CA=CAs[r % n], SCA=SCA, bitmap=bm)
+                ug = graph_us(torch, dev, st, one, reps)
+                row.update({"kernel_us": round(ug, 2), "kernel_GB/s": round(byts / ug / 1e3, 1),
+                            "kernel_frac": round(byts / ug / 1e3 / hbm, 4),
+                            "eager_us": round(us, 2), "eager_frac": round(gbs / hbm, 4)})
+            else:
+                row.update({"op_tau6_us": round(us, 2), "op_tau6_GB/s": round(gbs, 1),
+                            "op_tau6_frac": round(gbs / hbm, 4)})
         res.append(row)
         del Xs, CAs
     return {"kernel": "k_quant_rows", "peak_gbs": hbm,
             "peak_source": "of measured hbm_gbs" if measured_peaks() else "of fallback",
             "bytes": "2MK + MK + 4M + K/8 per call",
-            "timing": f"CUDA events over {reps} back-to-back calls, inputs rotated over > 2 x L2",
-            "kernel_us": "threshold 0: the quantiser kernel alone; op_tau6: memset + quantiser + column zeroing",
+            "timing": f"CUDA events over {reps} calls, inputs rotated over > 2 x L2; kernel_us: threshold 0, "
+                      "the quantiser kernel alone, the calls replayed from one CUDA graph; eager_us: the same "
+                      "calls issued from Python (host-bound); op_tau6_us: eager memset + quantiser + column "
+                      "zeroing",
             "points": res}
 
 
@@ -358,7 +401,8 @@ def measure_backward(i8, torch, dev, st, world, dist, reps: int = 20):
     """Input gradient through the frozen int8 layer for the distinct weight shapes of the
     Llama-7B-shaped layer at 4096 tokens: the transposed dequantisation of the weight
     (HBM-bound, 3NK bytes) and dX = dY . W^ on the fp16 tensor cores (2MNK flops), each
-    timed alone with CUDA events over `reps` back-to-back calls."""
+    timed alone with CUDA events over `reps` back-to-back calls (the dequantisation, shorter
+    than its host call, from a CUDA graph of `reps` calls; dequant_t_eager_us issued from Python)."""
     layers = wl.workloads()["C3"].layers
     peaks = measured_peaks()
     f16_peak = float(peaks["bf16_tflops"]) if peaks else 1590.0
@@ -387,13 +431,14 @@ def measure_backward(i8, torch, dev, st, world, dist, reps: int = 20):
         dY = torch.from_numpy(wl.grad_output(600 + li, L.M, L.N)).to(dev)
         Wt = torch.empty((L.K, L.N), dtype=torch.float16, device=dev)
         dX = torch.empty((L.M, L.K), dtype=torch.float16, device=dev)
-        us_dq = timed(lambda: i8.i8_dequant_transposed(CB, SCB, Wt))
+        us_dq_eager = timed(lambda: i8.i8_dequant_transposed(CB, SCB, Wt))
+        us_dq = graph_us(torch, dev, st, lambda: i8.i8_dequant_transposed(CB, SCB, Wt), reps)
         us_mm = timed(lambda: i8.i8_linear8bit_backward_input(dY, Wt, dX))
         gbs = 3.0 * L.N * L.K / us_dq / 1e3
         tflops = 2.0 * L.M * L.N * L.K / us_mm / 1e6
         points.append({"layer": L.name, "dY": f"{L.M}x{L.N}", "W": f"{L.N}x{L.K}",
                        "dequant_t_us": round(us_dq, 2), "dequant_t_GB/s": round(gbs, 1),
-                       "dequant_t_frac": round(gbs / hbm, 4),
+                       "dequant_t_frac": round(gbs / hbm, 4), "dequant_t_eager_us": round(us_dq_eager, 2),
                        "gemm_us": round(us_mm, 2), "gemm_TFLOP/s": round(tflops, 1),
                        "gemm_frac": round(tflops / f16_peak, 4)})
     return {"metric": "input-gradient fp16 GEMM TFLOP/s (2MNK/s) and transposed dequant GB/s",
@@ -518,16 +563,23 @@ def measure_other(i8, torch, dev, st, world, dist, reps: int = 50):
         # the two halves of the same forward, each timed alone: quantise + outlier preparation,
         # then the GEMM with its epilogue (it re-reads the prepared workspace)
         dX, CB, SCB, db, out, ws = a
-        us_prep = timed(lambda: i8.i8_linear8bit_prepare(dX, CB, L.threshold, ws, MAX_OUTLIER_COLS), n=20)
-        us_gemm = timed(lambda: i8.i8_linear8bit_matmul_dequant(CB, SCB, db, L.M, L.threshold, out, ws,
-                                                                 MAX_OUTLIER_COLS), n=20)
+        def prep():
+            i8.i8_linear8bit_prepare(dX, CB, L.threshold, ws, MAX_OUTLIER_COLS)
+
+        def gemm():
+            i8.i8_linear8bit_matmul_dequant(CB, SCB, db, L.M, L.threshold, out, ws, MAX_OUTLIER_COLS)
+        timed(prep, n=3)
+        us_prep = graph_us(torch, dev, st, prep, 20)
+        timed(gemm, n=3)
+        us_gemm = graph_us(torch, dev, st, gemm, 20)
         status(ws)
         points.append({"key": key, "threshold": L.threshold, "planted_cols": L.n_out,
                        "outlier_cols": n_cols, "us": round(us, 2), "TOPS": round(tops, 1),
                        "frac": round(tops / peak, 4), "prepare_us": round(us_prep, 2),
                        "gemm_us": round(us_gemm, 2)})
     res["llama13b_mlp_sweep"] = {"shape": "2048x5120->13824", "points": points,
-                                 "split": "prepare_us / gemm_us: the forward's two halves, each timed alone"}
+                                 "split": "prepare_us / gemm_us: the forward's two halves, each timed alone "
+                                          "(20 calls replayed from a CUDA graph)"}
     return res
 
 
@@ -912,15 +964,16 @@ def run_ours(args):
                                     f"{K} steps ({ms_instr / K:.4f} ms per instrumented step)",
                      "quant": None if quant is None else {
                          "kernel": quant["kernel"], "bytes": quant["bytes"], "peak_gbs": quant["peak_gbs"],
-                         "points": [[q["shape"], q["kernel_us"], q["kernel_GB/s"], q["kernel_frac"]]
+                         "points": [[q["shape"], q["kernel_us"], q["kernel_GB/s"], q["kernel_frac"], q["eager_us"]]
                                     for q in quant["points"]],
-                         "columns": ["shape", "us", "GB/s", "frac"]},
+                         "columns": ["shape", "us (graph)", "GB/s", "frac", "us (eager)"]},
                      "decode": None if decode is None else {
                          "kernel": "k_decode_prep + k_gemm_i8_decode (whole forward)", "bytes": decode["bytes"],
                          "peak_gbs": decode["peak_gbs"],
-                         "points": [[q["tokens"], q["outlier_cols"], q["shape"], q["us"], q["GB/s"], q["frac"]]
-                                    for q in decode["points"]],
-                         "columns": ["tokens", "outlier_cols", "shape", "us", "GB/s", "frac"]},
+                         "points": [[q["tokens"], q["outlier_cols"], q["shape"], q["us"], q["GB/s"], q["frac"],
+                                     q["us_graph"], q["frac_graph"]] for q in decode["points"]],
+                         "columns": ["tokens", "outlier_cols", "shape", "us", "GB/s", "frac", "us (graph)",
+                                     "frac (graph)"]},
                      "nf4": None if nf4 is None else {
                          "kernel": nf4["kernel"], "bytes": nf4["bytes"], "peak_gbs": nf4["peak_gbs"],
                          "points": [[q["shape"], q["us"], q["GB/s"], q["frac"]] for q in nf4["points"]],

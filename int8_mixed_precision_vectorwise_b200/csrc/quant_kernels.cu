@@ -230,17 +230,127 @@ __device__ __forceinline__ int outlier_slot(int pos) {
   return (pos & ~15) + 2 * (q >> 2) + (q & 1) + 8 * ((q >> 1) & 1);
 }
 
+// Stored position of list entry e in the gathered operands (the inverse of
+// outlier_slot).
+__device__ __forceinline__ int outlier_pos(int e) {
+  const int q = e & 15;
+  return (e & ~15) + 4 * ((q >> 1) & 3) + 2 * ((q >> 3) & 1) + (q & 1);
+}
+
+// With at least one listed column per kDenseRowBytes bytes of a weight row,
+// most 128-byte lines of every row hold a listed column and the scattered
+// gather is bound by its request count; reading the rows whole then costs
+// about the same DRAM bytes, in coalesced requests.
+constexpr int kDenseRowBytes = 48;
+// The dense preparation reads rows in batches of kDenseChunks chunks of 512 bytes (one
+// 16-byte load per lane and chunk); the list is indexed by 256-column chunks.
+constexpr int kDenseChunk = 512;
+constexpr int kDenseChunks = 8;  // chunks per batch
+constexpr int kDenseBatch = kDenseChunks * kDenseChunk;
+constexpr int kListChunkCols = 256;
+
+// Dynamic shared memory of the preparation: the list (cap entries), then, when
+// the dense mode can be taken, the chunk index (K / 256 + 1 entries) and two
+// 512-byte staging buffers per warp.
+__host__ __device__ inline size_t dense_stage_offset(int cap, int K) {
+  const size_t words = static_cast<size_t>(cap > 0 ? cap : 1) + (K + kListChunkCols - 1) / kListChunkCols + 1;
+  return (words * sizeof(int32_t) + 15) & ~static_cast<size_t>(15);
+}
+__host__ __device__ inline bool dense_possible(int cap, int K) {
+  return static_cast<long long>(cap) * kDenseRowBytes >= K;
+}
+
+__device__ __forceinline__ void load_batch(uint4 (&v)[kDenseChunks], const uint8_t* __restrict__ row, int b0, int row_bytes,
+                                           int lane) {
+#pragma unroll
+  for (int c = 0; c < kDenseChunks; ++c) {
+    const int off = b0 + c * kDenseChunk + lane * 16;
+    v[c] = off < row_bytes ? __ldcg(reinterpret_cast<const uint4*>(row + off)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The listed elements of one batch of a row (kEs bytes per element), starting
+// at byte b0.  Each 512-byte chunk goes through one of the warp's two staging
+// buffers (wbuf, 2 x 512 bytes); chunk c holds the list entries cst[x0] ..
+// cst[x1] - 1 (cst[x] = first entry at or past column 256 x), which the lanes
+// take 32 at a time.  X rows (kEs == 2) also zero their codes in ca.
+template <int kEs>
+__device__ __forceinline__ void take_batch(const uint4 (&v)[kDenseChunks], int b0, int row_bytes, const int32_t* idx_s,
+                                           const int32_t* cst, int n_cst, __half* __restrict__ dst,
+                                           int8_t* __restrict__ ca, uint8_t* wbuf, int lane) {
+#pragma unroll
+  for (int c = 0; c < kDenseChunks; ++c) {
+    const int lo = b0 + c * kDenseChunk;
+    if (lo >= row_bytes) break;
+    uint8_t* buf = wbuf + (c & 1) * kDenseChunk;
+    // the lanes finished the chunk before the previous one (the last reader of
+    // this buffer) before the __syncwarp of the previous chunk
+    *reinterpret_cast<uint4*>(buf + lane * 16) = v[c];
+    __syncwarp();
+    const int x0 = lo / (kEs * kListChunkCols);
+    const int x1 = min(x0 + kDenseChunk / (kEs * kListChunkCols), n_cst - 1);
+    const int e_hi = cst[x1];
+    for (int e = cst[x0] + lane; e < e_hi; e += 32) {
+      const int j = idx_s[e];
+      const int off = j * kEs - lo;
+      unsigned short h;
+      if (kEs == 2) {
+        h = *reinterpret_cast<const unsigned short*>(buf + off);
+        if (ca != nullptr) ca[j] = 0;
+      } else {
+        h = __half_as_ushort(__int2half_rn(static_cast<int>(reinterpret_cast<const int8_t*>(buf)[off])));
+      }
+      if (dst != nullptr) dst[outlier_pos(e)] = __ushort_as_half(h);
+    }
+  }
+  __syncwarp();  // the next batch starts again at buffer 0
+}
+
+// Rows first, first + stride, ... < rows of one operand, on one warp: the next
+// batch (of this row or the next) is requested before the current one is
+// taken apart.  dst / ca advance by ld_dst / row_elems per row (ca may be null,
+// dst too).  Positions used .. width - 1 of every dst row are zeroed.
+template <int kEs>
+__device__ __forceinline__ void prepare_rows_dense(const uint8_t* __restrict__ src, int row_elems, int rows,
+                                                   int first, int stride, const int32_t* idx_s, const int32_t* cst,
+                                                   int n_cst, int used, int width, __half* __restrict__ dst,
+                                                   int ld_dst, int8_t* __restrict__ ca, uint8_t* wbuf, int lane) {
+  const int row_bytes = row_elems * kEs;
+  const int nbat = (row_bytes + kDenseBatch - 1) / kDenseBatch;
+  int r = first, b = 0;
+  uint4 cur[kDenseChunks], nxt[kDenseChunks];
+  if (r < rows) load_batch(cur, src + static_cast<size_t>(r) * row_bytes, 0, row_bytes, lane);
+  while (r < rows) {
+    int r2 = r, b2 = b + 1;
+    if (b2 == nbat) {
+      r2 += stride;
+      b2 = 0;
+    }
+    if (r2 < rows) load_batch(nxt, src + static_cast<size_t>(r2) * row_bytes, b2 * kDenseBatch, row_bytes, lane);
+    __half* d = dst != nullptr ? dst + static_cast<size_t>(r) * ld_dst : nullptr;
+    take_batch<kEs>(cur, b * kDenseBatch, row_bytes, idx_s, cst, n_cst, d,
+                    ca != nullptr ? ca + static_cast<size_t>(r) * row_elems : nullptr, wbuf, lane);
+    if (b2 == 0 && d != nullptr)
+      for (int e = used + lane; e < width; e += 32) d[outlier_pos(e)] = __ushort_as_half(0);
+#pragma unroll
+    for (int c = 0; c < kDenseChunks; ++c) cur[c] = nxt[c];
+    r = r2;
+    b = b2;
+  }
+}
+
 // Outlier preparation for the fused forward.  Every block rebuilds the sorted
 // column list from the bitmap in shared memory (a block-wide scan of
-// popcounts); then the grid's threads take work items (row, group of 16 list
-// positions) over the X rows (gather X[:, O] into X_O, zero CA[:, O]) and the
-// CB rows (gather fp16(CB[:, O]) into W_O).  An item issues its 16 gathers at
-// once and writes the group as two 16-byte stores, so the scattered reads of
-// every (row, column) pair are in flight together across the grid.  Up to 16
-// used columns the operands are written as one zero-padded group of 16 (the
-// GEMM's epilogue reads exactly that); past 16, zero padded to a multiple of
-// 64 (one 128-byte fp16 tile of the tensor-core path).  Block 0 publishes the
-// list, the counts and the overflow status.
+// popcounts).  Then, with few listed columns, the grid's threads take work
+// items (row, group of 16 list positions) over the X rows (gather X[:, O] into
+// X_O, zero CA[:, O]) and the CB rows (gather fp16(CB[:, O]) into W_O): an item
+// issues its 16 gathers at once and writes the group as two 16-byte stores, so
+// the scattered reads of every (row, column) pair are in flight together across
+// the grid.  With many (see kDenseRowBytes), each warp streams whole rows
+// instead (prepare_row_dense).  Up to 16 used columns the operands are written
+// as one zero-padded group of 16 (the GEMM's epilogue reads exactly that); past
+// 16, zero padded to a multiple of 64 (one 128-byte fp16 tile of the tensor-core
+// path).  Block 0 publishes the list, the counts and the overflow status.
 __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restrict__ bitmap, int K, int cap,
                                                          int32_t* __restrict__ total_out,
                                                          int32_t* __restrict__ used_out,
@@ -305,6 +415,27 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
   const int groups = used <= 16 ? 1 : ((used + 63) & ~63) >> 4;  // 16-position groups written
   const int rows_x = (XO != nullptr || CA != nullptr) ? M : 0;
   const int rows_w = WO != nullptr ? N : 0;
+  if (rows_x + rows_w > 0 && static_cast<long long>(used) * kDenseRowBytes >= K) {
+    // cst[x] = first list entry at or past column 256 x, x = 0 .. n_cst - 1
+    int32_t* cst = idx_s + cap;
+    const int n_cst = (K + kListChunkCols - 1) / kListChunkCols + 1;
+    uint8_t* wbuf = reinterpret_cast<uint8_t*>(idx_s) + dense_stage_offset(cap, K) + warp * 2 * kDenseChunk;
+    for (int e = threadIdx.x; e <= used; e += 256) {
+      const int prev = e == 0 ? -1 : idx_s[e - 1] / kListChunkCols;  // chunk of the entry before
+      const int here = e == used ? n_cst - 1 : idx_s[e] / kListChunkCols;
+      for (int x = prev + 1; x <= here; ++x) cst[x] = e;
+    }
+    __syncthreads();
+    const int gw = blockIdx.x * 8 + warp, nw = gridDim.x * 8;
+    const int width = groups * 16;
+    if (rows_x > 0)
+      prepare_rows_dense<2>(reinterpret_cast<const uint8_t*>(X), K, rows_x, gw, nw, idx_s, cst, n_cst, used, width,
+                            XO, ld_o, CA, wbuf, lane);
+    if (rows_w > 0)
+      prepare_rows_dense<1>(reinterpret_cast<const uint8_t*>(CB), K, rows_w, gw, nw, idx_s, cst, n_cst, used, width,
+                            WO, ld_o, nullptr, wbuf, lane);
+    return;
+  }
   const long long items = static_cast<long long>(rows_x + rows_w) * groups;
   for (long long it = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; it < items;
        it += static_cast<long long>(gridDim.x) * 256) {
@@ -521,7 +652,8 @@ cudaError_t launch_outlier_prepare(const uint32_t* bitmap, int K, int cap, int32
   const int groups = cap <= 16 ? 1 : ((cap + 63) / 64) * 4;
   const long long items = static_cast<long long>(rows) * groups;
   const int blocks = static_cast<int>(std::max<long long>(1, std::min<long long>((items + 255) / 256, num_sms * 2LL)));
-  const size_t smem = static_cast<size_t>(max(cap, 1)) * sizeof(int32_t);
+  const size_t smem = rows > 0 && dense_possible(cap, K) ? dense_stage_offset(cap, K) + 8 * 2 * kDenseChunk
+                                                         : static_cast<size_t>(max(cap, 1)) * sizeof(int32_t);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks, 1, 1);
   cfg.blockDim = dim3(256, 1, 1);

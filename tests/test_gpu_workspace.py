@@ -145,6 +145,10 @@ PREP_CASES = [
     (4, 256, 28672, 5, 6.0, 64),       # 4 tokens on long rows: also the 16-CTA cluster
     (300, 520, 1040, 80, 6.0, 101),    # 80 columns, a capacity that is not a multiple of 4
     (260, 300, 8192, 100, 6.0, 256),   # 100 columns on long rows
+    # the preparation streams whole rows once there is a listed column per 48 bytes of row
+    (300, 520, 8192, 40, 6.0, 256),    # 40 columns on 8192-byte rows: gathered, padded to 64
+    (130, 264, 512, 12, 6.0, 256),     # 12 columns on 512-byte rows: streamed, one group of 16
+    (70, 136, 1040, 33, 6.0, 40),      # streamed, ragged last chunk, capacity 40 < 64
 ]
 
 
