@@ -54,6 +54,28 @@ constexpr int DS_BYTES = DT * DM * 4;      // one segment's outlier term, fp32 [
 constexpr int XS_COLS = 32;                // outlier columns of X[:, O] kept in shared memory
 constexpr int XS_BYTES = DT * XS_COLS * 2; // fp16 [column][token]
 
+// d[i][t] += X[t, j] * CB[row lane + 32 i, j] for tokens t < TT (>= T; the
+// rest of d is untouched), list entry c = column j at byte b of the 128-row
+// box `box` (128B swizzle: 16-byte chunk q of row r sits at q ^ (r % 8)).
+// X[:, j] comes from x_s ([column][token], zero past T) for the first XS_COLS
+// entries, else from X_O.
+template <int TT>
+__device__ __forceinline__ void outlier_column(float (&d)[4][kDecodeMaxTokens], const uint8_t* box, int b, int lane,
+                                               const __half* x_s, const __half* XO, int ld_o, int c, int T) {
+  float x[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t)
+    x[t] = c < XS_COLS ? __half2float(x_s[c * kDecodeMaxTokens + t])
+                       : (t < T ? __half2float(XO[static_cast<size_t>(t) * ld_o + c]) : 0.f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = lane + 32 * i;
+    const float w = static_cast<float>(static_cast<int8_t>(box[r * 128 + ((((b >> 4) ^ (r & 7))) << 4) + (b & 15)]));
+#pragma unroll
+    for (int t = 0; t < TT; ++t) d[i][t] = fmaf(x[t], w, d[i][t]);
+  }
+}
+
 template <int C>
 struct DecodeCfg {
   static constexpr int STAGE_BYTES = C * DBOX_BYTES;
@@ -294,19 +316,10 @@ __global__ void __launch_bounds__(DTHREADS, 1)
           if (j >= (k + 1) * DKS) break;
           const int kk = j - k * DKS;                // byte within the stage
           const int box = kk >> 7, b = kk & 127;     // 128-byte box, byte within the row
-          float x[DT];
-#pragma unroll
-          for (int t = 0; t < DT; ++t)
-            x[t] = cur < XS_COLS ? __half2float(x_s[cur * DT + t])
-                                 : (t < T ? __half2float(p.XO[static_cast<size_t>(t) * p.ld_o + cur]) : 0.f);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = lane + 32 * i;             // 128B swizzle: 16-byte chunk q of row r sits at q ^ (r % 8)
-            const float w = static_cast<float>(static_cast<int8_t>(
-                sa[box * DA_BYTES + r * 128 + ((((b >> 4) ^ (r & 7))) << 4) + (b & 15)]));
-#pragma unroll
-            for (int t = 0; t < DT; ++t) d[i][t] = fmaf(x[t], w, d[i][t]);
-          }
+          if (T <= 4)
+            outlier_column<4>(d, sa + box * DA_BYTES, b, lane, x_s, p.XO, p.ld_o, cur, T);
+          else
+            outlier_column<DT>(d, sa + box * DA_BYTES, b, lane, x_s, p.XO, p.ld_o, cur, T);
           ++cur;
         }
         __syncwarp();
