@@ -369,8 +369,15 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
   const int nwords = (K + 31) >> 5;
   const int per = (nwords + 255) / 256;
   const int w0 = min(threadIdx.x * per, nwords), w1 = min(w0 + per, nwords);
+  // up to 4 words per thread (K <= 32768) stay in registers for the second pass
+  uint32_t wv[4];
   int cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(__ldcg(bitmap + w));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    wv[q] = w0 + q < w1 ? __ldcg(bitmap + w0 + q) : 0u;
+    cnt += __popc(wv[q]);
+  }
+  for (int w = w0 + 4; w < w1; ++w) cnt += __popc(__ldcg(bitmap + w));
   int incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -390,15 +397,18 @@ __global__ void __launch_bounds__(256) k_outlier_prepare(const uint32_t* __restr
   }
   __syncthreads();
   int pos = warp_base[warp] + incl - cnt;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t bits = __ldcg(bitmap + w);
+  auto list_word = [&](int w, uint32_t bits) {  // the set bits of word w, in order
     while (bits) {
       const int b = __ffs(bits) - 1;
       bits &= bits - 1;
       if (pos < cap) idx_s[pos] = w * 32 + b;
       ++pos;
     }
-  }
+  };
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (w0 + q < w1) list_word(w0 + q, wv[q]);
+  for (int w = w0 + 4; w < w1; ++w) list_word(w, __ldcg(bitmap + w));
   __syncthreads();
   const int total = s_total;
   const int used = min(total, cap);
